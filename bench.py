@@ -1,0 +1,384 @@
+"""Benchmark of the Parallax hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload W]
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+  * decode  (headline, 1.7B-layer decode step): parallax_decode on B=64, H=16,
+    d=128 against a contiguous 4096-token bf16 KV cache -> HBM TB/s;
+  * prefill (1.7B-layer prefill): parallax_rho_proj (x [8,4096,2048] @ W_R
+    [2048,2048]) then parallax_fwd (B=8, T=4096, H=16, d=128, causal) -> TFLOP/s
+    counted as 8d flops per unmasked (i, j) pair (the four UMMAs).
+``value`` is the decode throughput; the prefill numbers ride in ``prefill``.
+All inputs are seeded synthetic data already resident in HBM; every input set
+is larger than the 126 MB L2, so no flush is needed between steps.
+
+The reference arm (--impl reference) times the fp64 CPU oracle on the host
+cores on a bounded sample of the same workloads and prints the same line.
+With N > 1 (torchrun) each rank runs an independent replica (the operator has
+no cross-GPU exchange); time is the max over ranks and value sums the ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Parallax attn: decode HBM TB/s, prefill TFLOP/s, % of roofline (1×B200)"
+DECODE_CFG = dict(B=64, H=16, Tcap=4096, d=128)
+PREFILL_CFG = dict(B=8, T=4096, H=16, d=128, d_model=2048)
+LONG_CFG = dict(B=1, T=32768, H=16, d=128, d_model=2048)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"],
+                "bf16_tflops_sustained": j.get("bf16_tflops_sustained"), "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def decode_bytes(B, H, d, seqlens):
+    """Algorithmic bytes of one decode call: K and V rows read + q, rho read + y (fp32) written."""
+    kv = int(np.sum(seqlens)) * H * d * 2 * 2
+    return kv + B * H * d * 2 * 2 + B * H * d * 4
+
+
+def prefill_pairs(B, H, T, causal=True):
+    return B * H * (T * (T + 1) // 2 if causal else T * T)
+
+
+def prefill_flops(B, H, T, d):
+    return 8 * d * prefill_pairs(B, H, T)
+
+
+def rho_proj_flops(B, T, d_model, H, d):
+    return 2 * B * T * d_model * H * d
+
+
+# --------------------------------------------------------------------------- #
+# clocks sampled during the timed region
+# --------------------------------------------------------------------------- #
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- #
+# our arm
+# --------------------------------------------------------------------------- #
+def run_ours(args, rank, world):
+    import torch
+
+    import softmax_learned_covariance_b200 as plx
+    from softmax_learned_covariance_b200 import inputs
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    peaks = load_peaks()
+
+    # ---------------- inputs (seeded, resident in HBM) ----------------
+    dc = DECODE_CFG
+    q, rho, kc, vc, sl = inputs.decode_inputs(dc["B"], dc["H"], dc["Tcap"], dc["d"], seed=2)
+    dq, drho, dk, dv = (t.torch().to(dev) for t in (q, rho, kc, vc))
+    dsl = torch.from_numpy(sl).to(dev)
+    yd = torch.empty((dc["B"], dc["H"], dc["d"]), dtype=torch.float32, device=dev)
+    d_bytes = decode_bytes(dc["B"], dc["H"], dc["d"], sl)
+    host_dec = [t.torch().pin_memory() for t in (q, rho, kc, vc)] + [torch.from_numpy(sl).pin_memory()]
+    del q, rho, kc, vc
+
+    pc = PREFILL_CFG if args.workload != "prefill_long" else LONG_CFG
+    x, w = inputs.rho_proj_inputs(pc["B"], pc["T"], pc["d_model"], pc["H"], pc["d"], seed=3)
+    pq, pk, pv, _ = inputs.fwd_bf16_inputs(pc["B"], pc["H"], pc["T"], pc["d"], seed=3)
+    dx, dw, dpq, dpk, dpv = (t.torch().to(dev) for t in (x, w, pq, pk, pv))
+    drho_p = torch.empty((pc["B"], pc["H"], pc["T"], pc["d"]), dtype=torch.bfloat16, device=dev)
+    yp = torch.empty((pc["B"], pc["H"], pc["T"], pc["d"]), dtype=torch.float32, device=dev)
+    lp = torch.empty((pc["B"], pc["H"], pc["T"]), dtype=torch.float32, device=dev)
+    host_pre = [t.torch().pin_memory() for t in (x, w, pq, pk, pv)]
+    del x, w, pq, pk, pv
+    p_flops = prefill_flops(pc["B"], pc["H"], pc["T"], pc["d"])
+    r_flops = rho_proj_flops(pc["B"], pc["T"], pc["d_model"], pc["H"], pc["d"])
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        plx.parallax_decode(dq, drho, dk, dv, dsl, y=yd, want_lse=False, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        plx.parallax_rho_proj(dx, dw, pc["H"], pc["d"], rho=drho_p, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        plx.parallax_fwd(dpq, dpk, dpv, drho_p, y=yp, lse=lp, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step()
+    assert plx.parallax_last_device_error() == 0
+    nsplit_units = plx.parallax_decode_workspace_bytes(dc["B"], dc["H"], dc["Tcap"], dc["d"])
+    launches_per_step = (2 if nsplit_units > 0 else 1) + 1 + 2
+
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    time.sleep(0.3)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    barrier()
+    clk = clocks.stop()
+    assert plx.parallax_last_device_error() == 0
+    total_ms = start.elapsed_time(end)
+    dec_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    rp_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    fwd_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
+
+    # max over ranks
+    vals = torch.tensor([total_ms, dec_ms, rp_ms, fwd_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    total_ms, dec_ms, rp_ms, fwd_ms = vals.tolist()
+
+    # ---------------- end to end through the public API, host buffers ----------------
+    e2e = e2e_pre = None
+    if not args.no_e2e:
+        ksteps = max(1, min(args.steps, 3))
+        h2d_d = sum(t.numel() * t.element_size() for t in host_dec)
+        d2h_d = yd.numel() * 4
+        yhost = torch.empty(yd.shape, dtype=torch.float32).pin_memory()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        t0.record(stream)
+        for _ in range(ksteps):
+            for dst, src in zip((dq, drho, dk, dv, dsl), host_dec):
+                dst.copy_(src, non_blocking=True)
+            plx.parallax_decode(dq, drho, dk, dv, dsl, y=yd, want_lse=False, stream=stream)
+            yhost.copy_(yd, non_blocking=True)
+        t1.record(stream)
+        barrier()
+        e_ms = t0.elapsed_time(t1)
+        e2e = {"value": world * d_bytes / (e_ms / ksteps * 1e-3) / 1e12, "unit": "TB/s",
+               "h2d_bytes_per_step": h2d_d, "d2h_bytes_per_step": d2h_d, "steps": ksteps}
+        h2d_p = sum(t.numel() * t.element_size() for t in host_pre)
+        yph = torch.empty(yp.shape, dtype=torch.float32).pin_memory()
+        barrier()
+        t0.record(stream)
+        for _ in range(ksteps):
+            for dst, src in zip((dx, dw, dpq, dpk, dpv), host_pre):
+                dst.copy_(src, non_blocking=True)
+            plx.parallax_rho_proj(dx, dw, pc["H"], pc["d"], rho=drho_p, stream=stream)
+            plx.parallax_fwd(dpq, dpk, dpv, drho_p, y=yp, lse=lp, stream=stream)
+            yph.copy_(yp, non_blocking=True)
+        t1.record(stream)
+        barrier()
+        e_ms = t0.elapsed_time(t1)
+        e2e_pre = {"value": world * (p_flops + r_flops) / (e_ms / ksteps * 1e-3) / 1e12, "unit": "TFLOP/s",
+                   "h2d_bytes_per_step": h2d_p, "d2h_bytes_per_step": yp.numel() * 4, "steps": ksteps}
+
+    dec_tbs = world * d_bytes / (dec_ms * 1e-3) / 1e12
+    fwd_tfs = world * p_flops / (fwd_ms * 1e-3) / 1e12
+    pre_tfs = world * (p_flops + r_flops) / ((fwd_ms + rp_ms) * 1e-3) / 1e12
+    rp_tfs = world * r_flops / (rp_ms * 1e-3) / 1e12
+    hbm = peaks["hbm_gbs"]
+    bf16 = peaks["bf16_tflops"]
+    tag = "of measured" if peaks["source"] == "measured" else "of fallback"
+    line = {
+        "metric": METRIC,
+        "value": round(dec_tbs, 4),
+        "unit": "TB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) q,k,v; rho ~ N(0,0.05^2) for decode; x ~ N(0,1), W_R ~ N(0,0.02^2) for prefill)",
+        "config": {"workload": "decode step B=64 H=16 d=128 ctx=4096 (headline) + prefill B=8 T=%d H=16 d=128 "
+                               "d_model=2048 causal" % pc["T"],
+                   "decode": dict(DECODE_CFG), "prefill": dict(pc), "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (2.1 GB decode cache, 0.6 GB prefill tensors); no flush"},
+        "roofline": {"bound": "hbm", "kernel": "parallax_decode (split + combine)", "achieved": round(dec_tbs * 1e3 / world, 1),
+                     "peak": hbm, "unit": "GB/s", "frac": round(dec_tbs * 1e3 / world / hbm, 4),
+                     "traffic": None, "peak_note": f"{tag} HBM copy bandwidth",
+                     "algorithmic_bytes_per_launch": d_bytes, "ms_per_launch": round(dec_ms, 5)},
+        "prefill": {"value": round(pre_tfs, 2), "unit": "TFLOP/s", "ms_per_step": round(fwd_ms + rp_ms, 4),
+                    "fwd": {"ms": round(fwd_ms, 4), "tflops": round(fwd_tfs / world, 2), "flops": p_flops,
+                            "roofline": {"bound": "tensor", "achieved": round(fwd_tfs / world, 2), "peak": bf16,
+                                         "unit": "TFLOP/s", "frac": round(fwd_tfs / world / bf16, 4),
+                                         "peak_note": f"{tag} dense bf16 (burst)"}},
+                    "rho_proj": {"ms": round(rp_ms, 4), "tflops": round(rp_tfs / world, 2), "flops": r_flops,
+                                 "frac": round(rp_tfs / world / bf16, 4)},
+                    "e2e": e2e_pre},
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+        "peaks": peaks,
+    }
+    return line
+
+
+# --------------------------------------------------------------------------- #
+# reference arm: the fp64 oracle on host cores, bounded samples of the same workloads
+# --------------------------------------------------------------------------- #
+def oracle_sample(budget_s=12.0):
+    import oracle
+    from softmax_learned_covariance_b200 import inputs
+
+    cores = oracle.max_threads()
+    dc = DECODE_CFG
+    # the first 4 sequences of the decode step (64 of its 1024 heads), same recipe and seed
+    nbs = 4
+    q, rho, kc, vc, sl = inputs.decode_inputs(nbs, dc["H"], dc["Tcap"], dc["d"], seed=2)
+    qf, rf, kf, vf = q.f64, rho.f64, kc.f64, vc.f64
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.decode(qf, rf, kf, vf, sl)
+        reps += 1
+        if time.perf_counter() - t0 > budget_s / 2:
+            break
+    dt = (time.perf_counter() - t0) / reps
+    dec_tbs = decode_bytes(nbs, dc["H"], dc["d"], sl) / dt / 1e12
+    dec_sample = f"{nbs * dc['H']} of the {dc['B'] * dc['H']} heads x {dc['Tcap']} tokens, x{reps}"
+
+    pc = PREFILL_CFG
+    pq, pk, pv, pr = inputs.fwd_bf16_inputs(1, 1, pc["T"], pc["d"], seed=3)
+    rows = np.arange(0, pc["T"], 8, dtype=np.int64)
+    t0 = time.perf_counter()
+    oracle.fwd_rows(pq.f64, pk.f64, pv.f64, pr.f64, rows)
+    dt = time.perf_counter() - t0
+    pairs = int(np.sum(rows + 1))
+    pre_tfs = 8 * pc["d"] * pairs / dt / 1e12
+    pre_sample = f"{rows.size} causal rows (every 8th) of one T={pc['T']} head, {pairs} pairs"
+    return cores, dec_tbs, dec_sample, pre_tfs, pre_sample
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    cores, dec_tbs, dec_sample, pre_tfs, pre_sample = oracle_sample()
+    line = {
+        "metric": METRIC, "value": dec_tbs, "unit": "TB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": "decode step B=64 H=16 d=128 ctx=4096 (headline) + prefill B=8 T=4096 H=16 d=128",
+                   "decode": dict(DECODE_CFG), "prefill": dict(PREFILL_CFG)},
+        "cpu_baseline": {"value": dec_tbs, "unit": "TB/s", "cores": cores, "kind": "oracle", "sample": dec_sample},
+        "prefill": {"value": pre_tfs, "unit": "TFLOP/s", "sample": pre_sample},
+        "e2e": {"value": dec_tbs, "unit": "TB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    return line
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["default", "prefill_long"], default="default")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world > 1 and args.impl == "ours":
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+    else:
+        line = run_ours(args, rank, world)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            cores, dec_tbs, dec_sample, _, _ = oracle_sample(budget_s=10.0)
+            line["cpu_baseline"] = {"value": dec_tbs, "unit": "TB/s", "cores": cores, "kind": "oracle",
+                                    "sample": dec_sample}
+    if rank == 0 and line is not None:
+        print(json.dumps(line), flush=True)
+    if world > 1 and args.impl == "ours":
+        import torch.distributed as dist
+
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,165 @@
+/*
+ * parallax.h -- C ABI of the Parallax attention library (B200, sm_100a).
+ *
+ * Parallax keeps exact softmax attention and subtracts the softmax-weighted
+ * key/value covariance projected by a learned probe rho_i = W_R x_i
+ * (zubnet.ai news item on Parallax, paragraph 2; encorp.ai blog "Integraciones
+ * de IA personalizadas tras la atencion Parallax", section "Por que eliminar el
+ * solucionador de gradiente conjugado..."):
+ *
+ *   z_ij = q_i . k_j / sqrt(d),  s_ij = softmax_j(z_ij) over the visible keys
+ *   o_i  = sum_j s_ij v_j,  a_ij = k_j . rho_i,  abar_i = sum_j s_ij a_ij,
+ *   m_i  = sum_j s_ij a_ij v_j
+ *   y_i  = o_i - C_i rho_i = o_i - (m_i - o_i abar_i)
+ *
+ * With rho = 0 (W_R = 0) the result is plain softmax attention exactly (same
+ * passages, and the encorp.ai FAQ on converting a pretrained Transformer).
+ *
+ * Conventions for every call:
+ *   - Tensors are caller-owned, contiguous, row-major DEVICE memory unless a
+ *     parameter says otherwise.  The library never frees or keeps them.
+ *   - Every device pointer must be 16-byte aligned (TMA and 128-bit loads).
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls only
+ *     enqueue work on it and return; results are ready when the stream is.
+ *   - A host-detectable error (null pointer, bad size, misalignment, an
+ *     unsupported dtype pair) returns a nonzero parallax_status_t and enqueues
+ *     nothing.  A failed launch returns PARALLAX_ERR_CUDA.  The library never
+ *     prints, never aborts and never falls back to another implementation.
+ *   - Device-side waits are bounded.  A wait that gives up records
+ *     PARALLAX_ERR_DEVICE_TIMEOUT in a per-device error word and the kernel
+ *     returns; read it with parallax_last_device_error().
+ *   - The library keeps one grow-only scratch allocation per device (the fp16
+ *     copy of V for the prefill kernel, the split partials for decode).  It
+ *     grows with cudaMalloc on first use, so the first call at a new, larger
+ *     size must not be inside CUDA graph capture.
+ */
+#ifndef PARALLAX_H
+#define PARALLAX_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define PARALLAX_API __attribute__((visibility("default")))
+#else
+#define PARALLAX_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void *parallax_stream_t; /* a cudaStream_t */
+
+typedef enum {
+    PARALLAX_F32 = 0,  /* IEEE binary32 */
+    PARALLAX_BF16 = 1  /* bfloat16 */
+} parallax_dtype_t;
+
+typedef enum {
+    PARALLAX_OK = 0,
+    PARALLAX_ERR_NULL = 1,           /* a required pointer is NULL */
+    PARALLAX_ERR_SHAPE = 2,          /* a size is out of range */
+    PARALLAX_ERR_ALIGN = 3,          /* a pointer is not 16-byte aligned */
+    PARALLAX_ERR_DTYPE = 4,          /* unsupported dtype or dtype pair */
+    PARALLAX_ERR_UNSUPPORTED = 5,    /* valid request this build does not serve */
+    PARALLAX_ERR_CUDA = 6,           /* a CUDA runtime/driver call failed */
+    PARALLAX_ERR_DEVICE_TIMEOUT = 7  /* a device-side wait gave up */
+} parallax_status_t;
+
+/*
+ * parallax_fwd -- prefill / forward over whole sequences.
+ *
+ * Passage: zubnet.ai news item on Parallax, paragraph 2 (output = softmax
+ * attention minus the probe-projected KV covariance; both branches reuse one
+ * KV stream); encorp.ai blog, section "Como cambia Parallax la historia del
+ * hardware en GPU Hopper" (same KV streaming structure as FlashAttention).
+ *
+ *   q, k, v, rho : [B, H, T, d] of in_dtype.  rho == NULL selects the
+ *                  softmax-only instantiation of the same kernel (y = o); with
+ *                  rho all zeros the result is bitwise equal to that.
+ *   y            : [B, H, T, d] of out_dtype (written).
+ *   lse          : [B, H, T] fp32, natural-log log-sum-exp of the scaled scores
+ *                  z_ij of each row (written); may be NULL.
+ *   B, H >= 1; T >= 1; d in {64, 128}.
+ *   causal       : nonzero -> query i sees keys 0..i; zero -> all T keys.
+ *   in_dtype/out_dtype:
+ *     F32  -> F32   fp32 CUDA-core kernel (fp32 arithmetic throughout)
+ *     BF16 -> F32   tensor-core kernel (tcgen05), fp32 accumulation
+ *     BF16 -> BF16  same kernel, y rounded to bf16 on store
+ *   Tensor-core path constraints: d == 128, |k_j . rho_i| < 65504 (the
+ *   correction weights are staged in fp16), |v| < 65504.
+ */
+PARALLAX_API int parallax_fwd(const void *q, const void *k, const void *v, const void *rho,
+                 void *y, float *lse, int B, int H, int T, int d, int causal,
+                 int in_dtype, int out_dtype, parallax_stream_t stream);
+
+/*
+ * parallax_decode -- one new query token per sequence against a KV cache.
+ *
+ * Passage: zubnet.ai news item on Parallax, paragraph 2 (the KV cache is still
+ * required for decoding; the decode kernel reuses one KV stream for both
+ * branches, which doubles the arithmetic intensity).
+ *
+ *   q, rho         : [B, H, d] bf16 (the current token's query and probe).
+ *   kcache, vcache : [B, H, Tcap, d] bf16; rows 0..seqlens[b]-1 are valid and
+ *                    already include the current token's key and value.
+ *   seqlens        : DEVICE int32 [B], 0 <= seqlens[b] <= Tcap (not read on the
+ *                    host; an empty sequence yields y = 0, lse = -inf).
+ *   y              : [B, H, d] of out_dtype (F32 or BF16).
+ *   lse            : [B, H] fp32, may be NULL.
+ *   B, H >= 1; Tcap >= 1; d in {64, 128}; in_dtype must be BF16.
+ * Uses the library's scratch for split partials; see parallax_decode_ex.
+ */
+PARALLAX_API int parallax_decode(const void *q, const void *rho, const void *kcache, const void *vcache,
+                    const int *seqlens, void *y, float *lse, int B, int H, int Tcap, int d,
+                    int in_dtype, int out_dtype, parallax_stream_t stream);
+
+/* Bytes of scratch parallax_decode_ex needs for this shape (0 if it needs none). */
+PARALLAX_API size_t parallax_decode_workspace_bytes(int B, int H, int Tcap, int d);
+
+/*
+ * parallax_decode_ex -- parallax_decode with caller-provided scratch.
+ *   workspace : device memory of at least parallax_decode_workspace_bytes(...)
+ *               bytes, 256-byte aligned, not used concurrently by another call.
+ *   Other arguments as parallax_decode.
+ */
+PARALLAX_API int parallax_decode_ex(const void *q, const void *rho, const void *kcache, const void *vcache,
+                       const int *seqlens, void *y, float *lse, int B, int H, int Tcap, int d,
+                       int in_dtype, int out_dtype, void *workspace, size_t workspace_bytes,
+                       parallax_stream_t stream);
+
+/*
+ * parallax_rho_proj -- the learned probe rho = x W_R, split per head.
+ *
+ * Passage: encorp.ai blog, section "Por que eliminar el solucionador de
+ * gradiente conjugado..." (a learned projector W_R acting on the layer input
+ * replaces the per-query solve); zubnet.ai, paragraph 2 (rho_i = W_R x_i).
+ *
+ *   x   : [B, T, d_model] bf16 (the layer input).
+ *   W_R : [d_model, H*d] bf16 row-major (column block h*d..h*d+d-1 is head h).
+ *   rho : [B, H, T, d] bf16 (written): rho[b,h,t,:] = x[b,t,:] @ W_R[:, h*d:(h+1)*d],
+ *         fp32 accumulation, rounded to bf16 on store.  No bias.
+ *   d_model % 64 == 0; (H*d) % 256 == 0; d in {64, 128}; dtype must be BF16.
+ */
+PARALLAX_API int parallax_rho_proj(const void *x, const void *W_R, void *rho, int B, int T, int d_model,
+                      int H, int d, int dtype, parallax_stream_t stream);
+
+/* Static English text for a status code (never NULL). */
+PARALLAX_API const char *parallax_strerror(int status);
+
+/*
+ * Synchronizes `stream`, then returns and clears the device error word of the
+ * current device: PARALLAX_OK, or PARALLAX_ERR_DEVICE_TIMEOUT when a kernel
+ * gave up on a bounded wait since the last read.  Returns PARALLAX_ERR_CUDA if
+ * the synchronization itself fails.
+ */
+PARALLAX_API int parallax_last_device_error(parallax_stream_t stream);
+
+/* Number of SMs the library sizes its persistent grids for on the current device (0 on error). */
+PARALLAX_API int parallax_device_sm_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PARALLAX_H */

@@ -1,0 +1,271 @@
+// api.cu -- the C ABI declared in include/parallax.h.
+//
+// Host side only: argument validation, per-device state (device error word,
+// grow-only scratch), TMA descriptor encoding and kernel launches.  Every
+// compute step runs in the CUDA kernels of this directory; there is no host
+// fallback.
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "internal.h"
+#include "parallax.h"
+
+using namespace plx;
+
+namespace {
+
+constexpr int MAX_DEVICES = 64;
+
+struct DevState {
+    bool init = false;
+    int sms = 0;
+    int *err = nullptr;
+    void *ws = nullptr;
+    size_t ws_bytes = 0;
+};
+
+std::mutex g_mu;
+DevState g_dev[MAX_DEVICES];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int status_of(cudaError_t e) { return e == cudaSuccess ? PARALLAX_OK : PARALLAX_ERR_CUDA; }
+
+int get_state(DevState **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return PARALLAX_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DevState &s = g_dev[dev];
+    if (!s.init) {
+        if (cudaDeviceGetAttribute(&s.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return PARALLAX_ERR_CUDA;
+        if (cudaMalloc(&s.err, sizeof(int)) != cudaSuccess) return PARALLAX_ERR_CUDA;
+        if (cudaMemset(s.err, 0, sizeof(int)) != cudaSuccess) return PARALLAX_ERR_CUDA;
+        s.init = true;
+    }
+    *out = &s;
+    return PARALLAX_OK;
+}
+
+// Grow-only scratch; the old buffer is released after the device is idle.
+int get_workspace(DevState *s, size_t bytes, void **out) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (bytes == 0) {
+        *out = s->ws;
+        return PARALLAX_OK;
+    }
+    if (s->ws_bytes < bytes) {
+        if (s->ws) {
+            if (cudaDeviceSynchronize() != cudaSuccess) return PARALLAX_ERR_CUDA;
+            cudaFree(s->ws);
+            s->ws = nullptr;
+            s->ws_bytes = 0;
+        }
+        const size_t want = (bytes + (1u << 20) - 1) & ~(size_t)((1u << 20) - 1);
+        if (cudaMalloc(&s->ws, want) != cudaSuccess) return PARALLAX_ERR_CUDA;
+        s->ws_bytes = want;
+    }
+    *out = s->ws;
+    return PARALLAX_OK;
+}
+
+DeviceCtl make_ctl(const DevState *s) {
+    DeviceCtl c;
+    c.err = s->err;
+    unsigned long long ms = 2000;
+    if (const char *e = std::getenv("PARALLAX_WAIT_TIMEOUT_MS")) {
+        const long v = std::strtol(e, nullptr, 10);
+        if (v > 0) ms = (unsigned long long)v;
+    }
+    c.wait_ns = ms * 1000000ull;
+    c.debug_flags = 0;
+    if (const char *e = std::getenv("PARALLAX_DEBUG_FLAGS")) c.debug_flags = (unsigned)std::strtoul(e, nullptr, 0);
+    return c;
+}
+
+int ensure_encoder() {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_encode) return PARALLAX_OK;
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return PARALLAX_ERR_CUDA;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    return PARALLAX_OK;
+}
+
+// Row-major tensor seen as up to 3 dims (inner first), 128-byte swizzled boxes.
+int encode(CUtensorMap *m, CUtensorMapDataType dt, const void *base, int rank, const uint64_t *dims,
+           const uint32_t *box, uint32_t elem_bytes) {
+    cuuint64_t gdim[3], gstride[2];
+    cuuint32_t gbox[3], estr[3] = {1, 1, 1};
+    uint64_t stride = elem_bytes;
+    for (int i = 0; i < rank; ++i) {
+        gdim[i] = dims[i];
+        gbox[i] = box[i];
+        if (i > 0) gstride[i - 1] = stride;
+        stride *= dims[i];
+    }
+    CUresult r = g_encode(m, dt, (cuuint32_t)rank, const_cast<void *>(base), gdim, gstride, gbox, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? PARALLAX_OK : PARALLAX_ERR_CUDA;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+const char *parallax_strerror(int status) {
+    switch (status) {
+        case PARALLAX_OK: return "ok";
+        case PARALLAX_ERR_NULL: return "a required pointer is NULL";
+        case PARALLAX_ERR_SHAPE: return "a size argument is out of range";
+        case PARALLAX_ERR_ALIGN: return "a pointer is not suitably aligned (16 bytes for tensors)";
+        case PARALLAX_ERR_DTYPE: return "unsupported dtype or dtype combination";
+        case PARALLAX_ERR_UNSUPPORTED: return "request not served by this build";
+        case PARALLAX_ERR_CUDA: return "a CUDA call failed";
+        case PARALLAX_ERR_DEVICE_TIMEOUT: return "a device-side wait gave up (bounded wait expired)";
+        default: return "unknown status";
+    }
+}
+
+int parallax_device_sm_count(void) {
+    DevState *s = nullptr;
+    if (get_state(&s) != PARALLAX_OK) return 0;
+    return s->sms;
+}
+
+int parallax_last_device_error(parallax_stream_t stream) {
+    DevState *s = nullptr;
+    int st = get_state(&s);
+    if (st) return st;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return PARALLAX_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, s->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return PARALLAX_ERR_CUDA;
+    if (v != 0 && cudaMemset(s->err, 0, sizeof(int)) != cudaSuccess) return PARALLAX_ERR_CUDA;
+    return v;
+}
+
+int parallax_fwd(const void *q, const void *k, const void *v, const void *rho, void *y, float *lse, int B, int H,
+                 int T, int d, int causal, int in_dtype, int out_dtype, parallax_stream_t stream) {
+    if (!q || !k || !v || !y) return PARALLAX_ERR_NULL;
+    if (B < 1 || H < 1 || T < 1 || (d != 64 && d != 128)) return PARALLAX_ERR_SHAPE;
+    if ((long long)B * H * T * d > (1ll << 40) || (long long)B * H > (1ll << 30)) return PARALLAX_ERR_SHAPE;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(y) || (rho && !aligned16(rho)) ||
+        (lse && !aligned4(lse)))
+        return PARALLAX_ERR_ALIGN;
+    const bool f32 = in_dtype == PARALLAX_F32 && out_dtype == PARALLAX_F32;
+    const bool bf16 = in_dtype == PARALLAX_BF16 && (out_dtype == PARALLAX_F32 || out_dtype == PARALLAX_BF16);
+    if (!f32 && !bf16) return PARALLAX_ERR_DTYPE;
+    if (bf16 && d != 128) return PARALLAX_ERR_UNSUPPORTED;
+
+    DevState *s = nullptr;
+    int st = get_state(&s);
+    if (st) return st;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+
+    if (f32) return status_of(launch_fwd_simt(q, k, v, rho, y, lse, B, H, T, d, causal, in_dtype, out_dtype, cs));
+
+    if ((st = ensure_encoder())) return st;
+    const size_t n = (size_t)B * H * T * d;
+    void *v16 = nullptr;
+    if ((st = get_workspace(s, n * 2, &v16))) return st;
+    if (launch_convert_bf16_to_f16(v, v16, n, cs) != cudaSuccess) return PARALLAX_ERR_CUDA;
+
+    FwdTensorMaps tm;
+    const uint64_t dims[3] = {(uint64_t)d, (uint64_t)T, (uint64_t)B * H};
+    const uint32_t box_q[3] = {64, 128, 1}, box_k[3] = {64, 64, 1};
+    if ((st = encode(&tm.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, 3, dims, box_q, 2))) return st;
+    if ((st = encode(&tm.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k, 3, dims, box_k, 2))) return st;
+    if ((st = encode(&tm.v16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, v16, 3, dims, box_k, 2))) return st;
+    if (rho) {
+        if ((st = encode(&tm.r, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rho, 3, dims, box_q, 2))) return st;
+    } else {
+        tm.r = tm.q;
+    }
+    return status_of(
+        launch_fwd_sm100(tm, rho != nullptr, y, lse, B, H, T, d, causal, out_dtype, s->sms, make_ctl(s), cs));
+}
+
+size_t parallax_decode_workspace_bytes(int B, int H, int Tcap, int d) {
+    if (B < 1 || H < 1 || Tcap < 1 || (d != 64 && d != 128)) return 0;
+    DevState *s = nullptr;
+    if (get_state(&s) != PARALLAX_OK) return 0;
+    return decode_partials_bytes(B, H, d, plan_decode(B, H, Tcap, d, s->sms));
+}
+
+static int decode_impl(const void *q, const void *rho, const void *kcache, const void *vcache, const int *seqlens,
+                       void *y, float *lse, int B, int H, int Tcap, int d, int in_dtype, int out_dtype,
+                       void *workspace, size_t workspace_bytes, bool own_workspace, parallax_stream_t stream) {
+    if (!q || !rho || !kcache || !vcache || !seqlens || !y) return PARALLAX_ERR_NULL;
+    if (B < 1 || H < 1 || Tcap < 1 || (d != 64 && d != 128)) return PARALLAX_ERR_SHAPE;
+    if ((long long)B * H * Tcap * d > (1ll << 40)) return PARALLAX_ERR_SHAPE;
+    if (!aligned16(q) || !aligned16(rho) || !aligned16(kcache) || !aligned16(vcache) || !aligned4(seqlens) ||
+        !aligned16(y) || (lse && !aligned4(lse)))
+        return PARALLAX_ERR_ALIGN;
+    if (in_dtype != PARALLAX_BF16 || (out_dtype != PARALLAX_F32 && out_dtype != PARALLAX_BF16))
+        return PARALLAX_ERR_DTYPE;
+    DevState *s = nullptr;
+    int st = get_state(&s);
+    if (st) return st;
+    const DecodePlan plan = plan_decode(B, H, Tcap, d, s->sms);
+    const size_t need = decode_partials_bytes(B, H, d, plan);
+    void *ws = nullptr;
+    if (own_workspace) {
+        if ((st = get_workspace(s, need, &ws))) return st;
+    } else {
+        if (need > 0 && (!workspace)) return PARALLAX_ERR_NULL;
+        if (workspace_bytes < need) return PARALLAX_ERR_SHAPE;
+        if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return PARALLAX_ERR_ALIGN;
+        ws = workspace;
+    }
+    return status_of(launch_decode(q, rho, kcache, vcache, seqlens, y, lse, B, H, Tcap, d, out_dtype, plan,
+                                   static_cast<float *>(ws), static_cast<cudaStream_t>(stream)));
+}
+
+int parallax_decode(const void *q, const void *rho, const void *kcache, const void *vcache, const int *seqlens,
+                    void *y, float *lse, int B, int H, int Tcap, int d, int in_dtype, int out_dtype,
+                    parallax_stream_t stream) {
+    return decode_impl(q, rho, kcache, vcache, seqlens, y, lse, B, H, Tcap, d, in_dtype, out_dtype, nullptr, 0, true,
+                       stream);
+}
+
+int parallax_decode_ex(const void *q, const void *rho, const void *kcache, const void *vcache, const int *seqlens,
+                       void *y, float *lse, int B, int H, int Tcap, int d, int in_dtype, int out_dtype,
+                       void *workspace, size_t workspace_bytes, parallax_stream_t stream) {
+    return decode_impl(q, rho, kcache, vcache, seqlens, y, lse, B, H, Tcap, d, in_dtype, out_dtype, workspace,
+                       workspace_bytes, false, stream);
+}
+
+int parallax_rho_proj(const void *x, const void *W_R, void *rho, int B, int T, int d_model, int H, int d, int dtype,
+                      parallax_stream_t stream) {
+    if (!x || !W_R || !rho) return PARALLAX_ERR_NULL;
+    if (B < 1 || T < 1 || H < 1 || (d != 64 && d != 128) || d_model < 64 || d_model % 64 != 0 || (H * d) % 256 != 0)
+        return PARALLAX_ERR_SHAPE;
+    if ((long long)B * T > (1ll << 31) - 1 || (long long)d_model * H * d > (1ll << 40)) return PARALLAX_ERR_SHAPE;
+    if (!aligned16(x) || !aligned16(W_R) || !aligned16(rho)) return PARALLAX_ERR_ALIGN;
+    if (dtype != PARALLAX_BF16) return PARALLAX_ERR_DTYPE;
+    DevState *s = nullptr;
+    int st = get_state(&s);
+    if (st) return st;
+    if ((st = ensure_encoder())) return st;
+    CUtensorMap tx, tw;
+    const uint64_t dx[2] = {(uint64_t)d_model, (uint64_t)B * T};
+    const uint32_t bx[2] = {64, 128};
+    const uint64_t dw[2] = {(uint64_t)H * d, (uint64_t)d_model};
+    const uint32_t bw[2] = {64, 64};
+    if ((st = encode(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, 2, dx, bx, 2))) return st;
+    if ((st = encode(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W_R, 2, dw, bw, 2))) return st;
+    return status_of(launch_rho_proj(tx, tw, rho, B, T, d_model, H, d, s->sms, make_ctl(s),
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,341 @@
+// decode.cu -- split-KV decode of one query token per sequence (HBM-bound).
+//
+// The pages' decode kernel reuses one KV stream for both branches (zubnet.ai
+// news item on Parallax, paragraph 2; encorp.ai blog, section "Como cambia
+// Parallax la historia del hardware en GPU Hopper"): per cached token the
+// kernel reads k_j once and forms both z_j = q.k_j/sqrt(d) and a_j = k_j.rho,
+// then reads v_j once and accumulates both o and m.  Per token: 8d flops for
+// 4d bytes of K and V.
+//
+// Work is cut into units of (b, h, chunk of tokens).  A grid of at most a few
+// waves of CTAs strides over the units, so ragged sequence lengths balance
+// without a host-side read of seqlens.  Within a unit the tokens are taken in
+// sub-chunks of SUB: pass A streams K with 16-byte loads (one token row per
+// D/8 lanes, fully coalesced) and stages z, a in shared memory; the sub-chunk
+// max updates the running max (one rescale per sub-chunk, not per token);
+// pass B streams V and accumulates o and m in fp32.  A unit writes either the
+// final y (one unit per sequence) or its partial state (mu, l, abar, O, M) for
+// the combine kernel, which merges the partials with max-rescaling.
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "internal.h"
+
+namespace plx {
+namespace {
+
+constexpr int NW = 8;          // warps per CTA
+constexpr int NTHREADS = NW * 32;
+constexpr int SUB = 512;       // tokens staged per sub-chunk
+constexpr int UNROLL = 4;      // loads in flight per lane per pass step
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr float LN2 = 0.6931471805599453f;
+
+__device__ __forceinline__ float fex2(float x) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ uint4 ldg_stream(const uint4 *p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8]) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        f[2 * t] = __uint_as_float(w[t] << 16);
+        f[2 * t + 1] = __uint_as_float(w[t] & 0xFFFF0000u);
+    }
+}
+
+template <typename Tout> __device__ __forceinline__ void store_out(Tout *p, float v);
+template <> __device__ __forceinline__ void store_out<float>(float *p, float v) { *p = v; }
+template <> __device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat16 *p, float v) {
+    *p = __float2bfloat16_rn(v);
+}
+
+template <int D> struct DecodeSmem {
+    static constexpr int LPT = D / 8;        // lanes per token row
+    static constexpr int TPW = 32 / LPT;     // token rows per warp step
+    static constexpr int GROUPS = NW * TPW;  // token slots per CTA step
+    float z[SUB];                            // scores (log2 units), then p
+    float a[SUB];                            // a_j, then p_j a_j
+    float red_o[GROUPS][D];
+    float red_m[GROUPS][D];
+    float red_s[3][NW];
+};
+
+template <int D, typename Tout>
+__global__ void __launch_bounds__(NTHREADS) k_decode_split(
+    const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ rho, const __nv_bfloat16 *__restrict__ kc,
+    const __nv_bfloat16 *__restrict__ vc, const int *__restrict__ seqlens, Tout *__restrict__ y,
+    float *__restrict__ lse, int H, int Tcap, int chunk, int nsplit, long units, float *__restrict__ partials) {
+    using S = DecodeSmem<D>;
+    constexpr int LPT = S::LPT, TPW = S::TPW, GROUPS = S::GROUPS;
+    constexpr int STEP = GROUPS * UNROLL;    // token rows per unrolled step
+    __shared__ S sm;
+
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    const int g = lane / LPT;                 // token slot within the warp
+    const int c = lane % LPT;                 // 16-byte column within the row
+    const int slot = warp * TPW + g;          // token slot within the CTA step
+    const float scale_log2 = LOG2E / sqrtf((float)D);
+
+    for (long u = blockIdx.x; u < units; u += gridDim.x) {
+        const long bh = u / nsplit;
+        const int split = (int)(u % nsplit);
+        const int b = (int)(bh / H);
+        const int L = min(max(seqlens[b], 0), Tcap);   // never read past the cache
+        const int t0 = split * chunk;
+        if (t0 >= L && nsplit > 1) continue;  // beyond this sequence: no partial
+        const int t1 = min(L, t0 + chunk);
+
+        float qv[8], rv[8];
+        {
+            const uint4 *qp = reinterpret_cast<const uint4 *>(q + bh * D) + c;
+            const uint4 *rp = reinterpret_cast<const uint4 *>(rho + bh * D) + c;
+            unpack8(__ldg(qp), qv);
+            unpack8(__ldg(rp), rv);
+        }
+        const uint4 *kbase = reinterpret_cast<const uint4 *>(kc + (size_t)bh * Tcap * D) + c;
+        const uint4 *vbase = reinterpret_cast<const uint4 *>(vc + (size_t)bh * Tcap * D) + c;
+
+        float mu = -INFINITY, lsum = 0.f, asum = 0.f;
+        float O[8], M[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) O[e] = M[e] = 0.f;
+
+        for (int s0 = t0; s0 < t1; s0 += SUB) {
+            const int n = min(SUB, t1 - s0);
+            // ---- pass A: K stream -> z (log2 units) and a ----
+            for (int base = 0; base < n; base += STEP) {
+                uint4 kr[UNROLL];
+#pragma unroll
+                for (int x = 0; x < UNROLL; ++x) {
+                    const int tok = base + x * GROUPS + slot;
+                    kr[x] = tok < n ? ldg_stream(kbase + (size_t)(s0 + tok) * LPT) : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int x = 0; x < UNROLL; ++x) {
+                    float kf[8];
+                    unpack8(kr[x], kf);
+                    float dz = 0.f, da = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        dz = fmaf(qv[e], kf[e], dz);
+                        da = fmaf(rv[e], kf[e], da);
+                    }
+#pragma unroll
+                    for (int off = LPT / 2; off > 0; off >>= 1) {
+                        dz += __shfl_xor_sync(0xffffffffu, dz, off);
+                        da += __shfl_xor_sync(0xffffffffu, da, off);
+                    }
+                    const int tok = base + x * GROUPS + slot;
+                    if (c == 0 && tok < n) {
+                        sm.z[tok] = dz * scale_log2;
+                        sm.a[tok] = da;
+                    }
+                }
+            }
+            __syncthreads();
+            // ---- sub-chunk max, running rescale ----
+            float mx = -INFINITY;
+            for (int t = tid; t < n; t += NTHREADS) mx = fmaxf(mx, sm.z[t]);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            if (lane == 0) sm.red_s[0][warp] = mx;
+            __syncthreads();
+            mx = sm.red_s[0][0];
+#pragma unroll
+            for (int w = 1; w < NW; ++w) mx = fmaxf(mx, sm.red_s[0][w]);
+            const float mu_new = fmaxf(mu, mx);
+            const float alpha = fex2(mu - mu_new);   // 0 when mu = -inf
+            mu = mu_new;
+            lsum *= alpha;
+            asum *= alpha;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                O[e] *= alpha;
+                M[e] *= alpha;
+            }
+            for (int t = tid; t < n; t += NTHREADS) {
+                const float p = fex2(sm.z[t] - mu);
+                const float pa = p * sm.a[t];
+                sm.z[t] = p;
+                sm.a[t] = pa;
+                lsum += p;
+                asum += pa;
+            }
+            __syncthreads();
+            // ---- pass B: V stream -> O += p v, M += p a v ----
+            for (int base = 0; base < n; base += STEP) {
+                uint4 vr[UNROLL];
+#pragma unroll
+                for (int x = 0; x < UNROLL; ++x) {
+                    const int tok = base + x * GROUPS + slot;
+                    vr[x] = tok < n ? ldg_stream(vbase + (size_t)(s0 + tok) * LPT) : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int x = 0; x < UNROLL; ++x) {
+                    const int tok = base + x * GROUPS + slot;
+                    if (tok < n) {
+                        float vf[8];
+                        unpack8(vr[x], vf);
+                        const float p = sm.z[tok], pa = sm.a[tok];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            O[e] = fmaf(p, vf[e], O[e]);
+                            M[e] = fmaf(pa, vf[e], M[e]);
+                        }
+                    }
+                }
+            }
+            __syncthreads();
+        }
+
+        // ---- reduce over token slots and threads ----
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            sm.red_o[slot][c * 8 + e] = O[e];
+            sm.red_m[slot][c * 8 + e] = M[e];
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
+            asum += __shfl_xor_sync(0xffffffffu, asum, off);
+        }
+        if (lane == 0) {
+            sm.red_s[1][warp] = lsum;
+            sm.red_s[2][warp] = asum;
+        }
+        __syncthreads();
+        if (tid < D) {
+            float l = 0.f, ab = 0.f, o = 0.f, m = 0.f;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+                l += sm.red_s[1][w];
+                ab += sm.red_s[2][w];
+            }
+#pragma unroll
+            for (int s = 0; s < GROUPS; ++s) {
+                o += sm.red_o[s][tid];
+                m += sm.red_m[s][tid];
+            }
+            if (nsplit == 1) {
+                float out = 0.f;
+                if (l > 0.f) {
+                    const float inv = 1.0f / l;
+                    const float oo = o * inv;
+                    out = oo - (m * inv - oo * (ab * inv));
+                }
+                store_out<Tout>(y + bh * D + tid, out);
+                if (lse != nullptr && tid == 0) lse[bh] = l > 0.f ? (mu + log2f(l)) * LN2 : -INFINITY;
+            } else {
+                float *P = partials + ((size_t)bh * nsplit + split) * (2 * D + 3);
+                if (tid == 0) {
+                    P[0] = mu;
+                    P[1] = l;
+                    P[2] = ab;
+                }
+                P[3 + tid] = o;
+                P[3 + D + tid] = m;
+            }
+        }
+        __syncthreads();
+    }
+}
+
+template <int D, typename Tout>
+__global__ void __launch_bounds__(D) k_decode_combine(const float *__restrict__ partials,
+                                                      const int *__restrict__ seqlens, Tout *__restrict__ y,
+                                                      float *__restrict__ lse, int H, int chunk, int nsplit) {
+    const long bh = blockIdx.x;
+    const int b = (int)(bh / H);
+    const int L = min(max(seqlens[b], 0), chunk * nsplit);
+    const int nvalid = min(nsplit, (L + chunk - 1) / chunk);
+    const int t = threadIdx.x;
+    const float *P = partials + (size_t)bh * nsplit * (2 * D + 3);
+    if (nvalid <= 0) {
+        store_out<Tout>(y + bh * D + t, 0.f);
+        if (lse != nullptr && t == 0) lse[bh] = -INFINITY;
+        return;
+    }
+    float mu = -INFINITY;
+    for (int s = 0; s < nvalid; ++s) mu = fmaxf(mu, P[(size_t)s * (2 * D + 3)]);
+    float l = 0.f, ab = 0.f, o = 0.f, m = 0.f;
+    for (int s = 0; s < nvalid; ++s) {
+        const float *Ps = P + (size_t)s * (2 * D + 3);
+        const float w = fex2(Ps[0] - mu);
+        l = fmaf(w, Ps[1], l);
+        ab = fmaf(w, Ps[2], ab);
+        o = fmaf(w, Ps[3 + t], o);
+        m = fmaf(w, Ps[3 + D + t], m);
+    }
+    const float inv = 1.0f / l;
+    const float oo = o * inv;
+    store_out<Tout>(y + bh * D + t, oo - (m * inv - oo * (ab * inv)));
+    if (lse != nullptr && t == 0) lse[bh] = (mu + log2f(l)) * LN2;
+}
+
+template <int D, typename Tout>
+cudaError_t launch_t(const void *q, const void *rho, const void *kc, const void *vc, const int *seqlens, void *y,
+                     float *lse, int B, int H, int Tcap, const DecodePlan &p, float *partials, cudaStream_t s) {
+    const long units = (long)B * H * p.nsplit;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    long grid = units;
+    const long cap = (long)sms * 8;
+    if (grid > cap) grid = cap;
+    k_decode_split<D, Tout><<<(unsigned)grid, NTHREADS, 0, s>>>(
+        (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)rho, (const __nv_bfloat16 *)kc, (const __nv_bfloat16 *)vc,
+        seqlens, (Tout *)y, lse, H, Tcap, p.chunk, p.nsplit, units, partials);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || p.nsplit == 1) return e;
+    k_decode_combine<D, Tout><<<(unsigned)(B * H), D, 0, s>>>(partials, seqlens, (Tout *)y, lse, H, p.chunk,
+                                                              p.nsplit);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+DecodePlan plan_decode(int B, int H, int Tcap, int d, int sm_count) {
+    (void)d;
+    DecodePlan p;
+    const long bh = (long)B * H;
+    const long wave = (long)sm_count * 8;            // resident CTAs of 256 threads
+    const long want_units = 8 * wave;                // several units per CTA for balance
+    long chunk = ((long)Tcap * bh + want_units - 1) / want_units;
+    chunk = ((chunk + 255) / 256) * 256;
+    if (chunk < 256) chunk = 256;
+    if (chunk >= Tcap) chunk = Tcap;                 // one unit per sequence
+    p.chunk = (int)chunk;
+    p.nsplit = (int)(((long)Tcap + chunk - 1) / chunk);
+    return p;
+}
+
+size_t decode_partials_bytes(int B, int H, int d, const DecodePlan &p) {
+    if (p.nsplit <= 1) return 0;
+    return (size_t)B * H * p.nsplit * (2 * d + 3) * sizeof(float);
+}
+
+cudaError_t launch_decode(const void *q, const void *rho, const void *kc, const void *vc, const int *seqlens,
+                          void *y, float *lse, int B, int H, int Tcap, int d, int out_dtype, const DecodePlan &p,
+                          float *partials, cudaStream_t s) {
+    if (d == 64) {
+        if (out_dtype == PARALLAX_F32)
+            return launch_t<64, float>(q, rho, kc, vc, seqlens, y, lse, B, H, Tcap, p, partials, s);
+        return launch_t<64, __nv_bfloat16>(q, rho, kc, vc, seqlens, y, lse, B, H, Tcap, p, partials, s);
+    }
+    if (out_dtype == PARALLAX_F32)
+        return launch_t<128, float>(q, rho, kc, vc, seqlens, y, lse, B, H, Tcap, p, partials, s);
+    return launch_t<128, __nv_bfloat16>(q, rho, kc, vc, seqlens, y, lse, B, H, Tcap, p, partials, s);
+}
+
+}  // namespace plx

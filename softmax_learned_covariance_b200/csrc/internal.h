@@ -1,0 +1,50 @@
+// internal.h -- launch entry points shared between the host API and the kernels.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "parallax.h"
+
+namespace plx {
+
+// Per-launch wait policy: absolute %globaltimer deadline is computed in-kernel
+// from this budget (nanoseconds).
+struct DeviceCtl {
+    int *err;                       // device error word
+    unsigned long long wait_ns;     // bound for every device-side wait
+    unsigned int debug_flags;       // test hooks (see DEBUG_*), 0 in normal use
+};
+constexpr unsigned DEBUG_FWD_SKIP_FIRST_K_LOAD = 1u;   // fwd: never load the first K tile
+
+// V [rows, d] bf16 -> fp16 (the PV operand precision of the tensor-core forward)
+cudaError_t launch_convert_bf16_to_f16(const void *src, void *dst, size_t n, cudaStream_t s);
+
+// fp32 / bf16 CUDA-core forward (one warp per query row)
+cudaError_t launch_fwd_simt(const void *q, const void *k, const void *v, const void *rho, void *y, float *lse,
+                            int B, int H, int T, int d, int causal, int in_dtype, int out_dtype, cudaStream_t s);
+
+// split-KV decode + combine
+struct DecodePlan {
+    int nsplit;      // CTAs per (b,h)
+    int chunk;       // tokens per split (multiple of 64)
+};
+DecodePlan plan_decode(int B, int H, int Tcap, int d, int sm_count);
+size_t decode_partials_bytes(int B, int H, int d, const DecodePlan &p);
+cudaError_t launch_decode(const void *q, const void *rho, const void *kc, const void *vc, const int *seqlens,
+                          void *y, float *lse, int B, int H, int Tcap, int d, int out_dtype, const DecodePlan &p,
+                          float *partials, cudaStream_t s);
+
+// tcgen05 GEMM for rho = x W_R, scattered per head
+cudaError_t launch_rho_proj(const CUtensorMap &tm_x, const CUtensorMap &tm_w, void *rho, int B, int T, int d_model,
+                            int H, int d, int sm_count, const DeviceCtl &ctl, cudaStream_t s);
+
+// tcgen05 causal/full prefill forward, bf16 in, fp16 V copy, fp32 accumulate
+struct FwdTensorMaps {
+    CUtensorMap q, k, r, v16;
+};
+cudaError_t launch_fwd_sm100(const FwdTensorMaps &tm, bool with_rho, void *y, float *lse, int B, int H, int T,
+                             int d, int causal, int out_dtype, int sm_count, const DeviceCtl &ctl, cudaStream_t s);
+
+}  // namespace plx

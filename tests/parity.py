@@ -1,0 +1,54 @@
+"""Shared comparison helpers for the parity tests (no operator arithmetic here).
+
+Tolerances for the bf16 tensor-core path: per head, max abs error <= 2e-2 and
+relative Frobenius error ||y - y_ref||_F / ||y_ref||_F <= 5e-3, gated on the
+fp32 output; fp32 path: max abs error <= 1e-4.  lse: max abs error <= 1e-3.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+BF16_MAX_ABS = 2e-2
+BF16_REL_F = 5e-3
+F32_MAX_ABS = 1e-4
+LSE_MAX_ABS = 1e-3
+
+
+def head_errors(y, ref, head_axes):
+    """(max_abs, rel_f) arrays over the leading `head_axes` dims."""
+    y = np.asarray(y, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert y.shape == ref.shape, (y.shape, ref.shape)
+    lead = y.shape[:head_axes]
+    d = (y - ref).reshape(*lead, -1)
+    r = ref.reshape(*lead, -1)
+    max_abs = np.max(np.abs(d), axis=-1)
+    rel_f = np.linalg.norm(d, axis=-1) / np.maximum(np.linalg.norm(r, axis=-1), 1e-30)
+    return max_abs, rel_f
+
+
+def assert_bf16_parity(y, ref, head_axes=2, what=""):
+    assert np.all(np.isfinite(y)), f"{what}: non-finite output"
+    ma, rf = head_errors(y, ref, head_axes)
+    assert ma.max() <= BF16_MAX_ABS, f"{what}: worst head max abs {ma.max():.3e} > {BF16_MAX_ABS}"
+    assert rf.max() <= BF16_REL_F, f"{what}: worst head rel-F {rf.max():.3e} > {BF16_REL_F}"
+    return float(ma.max()), float(rf.max())
+
+
+def assert_f32_parity(y, ref, what=""):
+    assert np.all(np.isfinite(y)), f"{what}: non-finite output"
+    err = float(np.max(np.abs(np.asarray(y, np.float64) - ref)))
+    assert err <= F32_MAX_ABS, f"{what}: max abs {err:.3e} > {F32_MAX_ABS}"
+    return err
+
+
+def assert_lse(lse, ref, what=""):
+    err = float(np.max(np.abs(np.asarray(lse, np.float64) - ref)))
+    assert err <= LSE_MAX_ABS, f"{what}: lse max abs {err:.3e} > {LSE_MAX_ABS}"
+    return err
+
+
+def sample_rows(T, n_head_rows=64, stride=127):
+    """Deterministic row subset: first/last n rows and every `stride`-th row."""
+    rows = set(range(min(T, n_head_rows))) | set(range(max(0, T - n_head_rows), T)) | set(range(0, T, stride))
+    return np.array(sorted(rows), dtype=np.int64)

@@ -1,0 +1,89 @@
+"""C-ABI checks that need no GPU: the library loads, exports every declared entry
+point, and rejects bad arguments on the host before touching the device."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import softmax_learned_covariance_b200 as plx
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"PARALLAX_API\s+[\w\s\*]+?\b(parallax_\w+)\s*\(", src))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def L():
+    from softmax_learned_covariance_b200 import build
+
+    build.build()
+    return plx.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_symbols()
+    assert len(names) >= 8
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in include/ but not exported"
+
+
+def test_strerror_covers_all_codes(L):
+    for code in range(8):
+        s = plx.parallax_strerror(code)
+        assert s and s != "unknown status"
+    assert plx.parallax_strerror(99) == "unknown status"
+
+
+P = ctypes.c_void_p
+A16 = P(0x10000)      # fake, 16-byte aligned (never dereferenced: validation fails first)
+MIS = P(0x10008)      # fake, misaligned
+
+
+def fwd(L, q=A16, k=A16, v=A16, rho=A16, y=A16, lse=None, B=1, H=1, T=8, d=128, causal=1, i=1, o=0):
+    return L.parallax_fwd(q, k, v, rho, y, lse, B, H, T, d, causal, i, o, None)
+
+
+def test_fwd_host_validation(L):
+    assert fwd(L, q=None) == 1
+    assert fwd(L, y=None) == 1
+    assert fwd(L, T=0) == 2
+    assert fwd(L, d=96) == 2
+    assert fwd(L, B=-1) == 2
+    assert fwd(L, k=MIS) == 3
+    assert fwd(L, rho=MIS) == 3
+    assert fwd(L, lse=P(0x10002)) == 3
+    assert fwd(L, i=1, o=5) == 4
+    assert fwd(L, i=0, o=1) == 4
+    assert fwd(L, d=64, i=1, o=0) == 5      # bf16 tensor-core path needs d = 128
+
+
+def test_decode_host_validation(L):
+    def dec(q=A16, rho=A16, kc=A16, vc=A16, sl=A16, y=A16, B=2, H=2, Tcap=16, d=128, i=1, o=0):
+        return L.parallax_decode(q, rho, kc, vc, sl, y, None, B, H, Tcap, d, i, o, None)
+    assert dec(rho=None) == 1
+    assert dec(sl=None) == 1
+    assert dec(Tcap=0) == 2
+    assert dec(d=32) == 2
+    assert dec(kc=MIS) == 3
+    assert dec(i=0) == 4
+    assert dec(o=7) == 4
+
+
+def test_rho_proj_host_validation(L):
+    def rp(x=A16, w=A16, r=A16, B=1, T=4, dm=128, H=2, d=128, dt=1):
+        return L.parallax_rho_proj(x, w, r, B, T, dm, H, d, dt, None)
+    assert rp(x=None) == 1
+    assert rp(dm=100) == 2
+    assert rp(H=1, d=128) == 2           # H*d must be a multiple of 256
+    assert rp(w=MIS) == 3
+    assert rp(dt=0) == 4

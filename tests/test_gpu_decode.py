@@ -1,0 +1,85 @@
+"""Decode parity: split-KV CUDA kernels (through the C ABI) vs the fp64 oracle."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import softmax_learned_covariance_b200 as plx
+from softmax_learned_covariance_b200 import inputs
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def _run(q, rho, kc, vc, sl, out_dtype=torch.float32):
+    y, lse = plx.parallax_decode(q.torch().to(DEV), rho.torch().to(DEV), kc.torch().to(DEV), vc.torch().to(DEV),
+                                 torch.from_numpy(sl).to(DEV), out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert plx.parallax_last_device_error() == 0
+    return y, lse
+
+
+def test_config2_decode_step_full():
+    """B=64 H=16 d=128, contiguous cache of 4096 tokens: every head vs the oracle."""
+    q, rho, kc, vc, sl = inputs.decode_inputs(64, 16, 4096, 128, seed=2)
+    y, lse = _run(q, rho, kc, vc, sl)
+    yr, lr = oracle.decode(q.f64, rho.f64, kc.f64, vc.f64, sl)
+    parity.assert_bf16_parity(y.cpu().numpy(), yr, 2, "config2")
+    parity.assert_lse(lse.cpu().numpy(), lr, "config2 lse")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("Tcap", [1, 7, 64, 300, 1000, 5000])
+def test_ragged_lengths(Tcap, d):
+    B, H = 5, 3
+    rng = np.random.default_rng(Tcap + d)
+    sl = rng.integers(1, Tcap + 1, size=B).astype(np.int32)
+    sl[0] = 1
+    sl[-1] = Tcap
+    q, rho, kc, vc, _ = inputs.decode_inputs(B, H, Tcap, d, seqlens=sl, seed=Tcap)
+    y, lse = _run(q, rho, kc, vc, sl)
+    yr, lr = oracle.decode(q.f64, rho.f64, kc.f64, vc.f64, sl)
+    parity.assert_bf16_parity(y.cpu().numpy(), yr, 2, f"Tcap={Tcap} d={d}")
+    parity.assert_lse(lse.cpu().numpy(), lr)
+
+
+def test_empty_sequence_and_bf16_output():
+    B, H, Tcap, d = 4, 2, 600, 128
+    sl = np.array([0, 1, 599, 600], np.int32)
+    q, rho, kc, vc, _ = inputs.decode_inputs(B, H, Tcap, d, seqlens=sl, seed=44)
+    y, lse = _run(q, rho, kc, vc, sl)
+    yr, lr = oracle.decode(q.f64, rho.f64, kc.f64, vc.f64, sl)
+    yg = y.cpu().numpy()
+    assert np.all(yg[0] == 0.0) and np.all(np.isneginf(lse.cpu().numpy()[0]))
+    parity.assert_bf16_parity(yg[1:], yr[1:], 2, "nonempty")
+    y16, _ = _run(q, rho, kc, vc, sl, out_dtype=torch.bfloat16)
+    assert torch.equal(y16, y.to(torch.bfloat16))
+
+
+def test_decode_ex_caller_workspace_matches():
+    q, rho, kc, vc, sl = inputs.decode_inputs(8, 16, 8192, 128, seed=21)
+    dq, dr, dk, dv, ds = (t.to(DEV) for t in (q.torch(), rho.torch(), kc.torch(), vc.torch(), torch.from_numpy(sl)))
+    nbytes = plx.parallax_decode_workspace_bytes(8, 16, 8192, 128)
+    ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=DEV)
+    y1, l1 = plx.parallax_decode(dq, dr, dk, dv, ds)
+    y2, l2 = plx.parallax_decode_ex(dq, dr, dk, dv, ds, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2) and torch.equal(l1, l2)
+    if nbytes > 0:
+        with pytest.raises(plx.ParallaxError):
+            plx.parallax_decode_ex(dq, dr, dk, dv, ds, ws[: nbytes // 2])
+
+
+def test_sweep_cell_sampled_heads():
+    """One mid-size cell of the decode sweep (B=64, context 8192, ragged), sampled heads."""
+    B, H, ctx, d = 64, 16, 8192, 128
+    sl = inputs.ragged_seqlens(B, ctx, seed=4 + 13)
+    q, rho, kc, vc, _ = inputs.decode_inputs(B, H, ctx, d, seqlens=sl, seed=4 + 13)
+    y, lse = _run(q, rho, kc, vc, sl)
+    bh = np.arange(0, B * H, 37)
+    yr, lr = oracle.decode(q.f64, rho.f64, kc.f64, vc.f64, sl, bh_list=bh)
+    parity.assert_bf16_parity(y.cpu().numpy().reshape(B * H, d)[bh], yr, 1, "sweep cell")
+    parity.assert_lse(lse.cpu().numpy().reshape(-1)[bh], lr)

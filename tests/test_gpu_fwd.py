@@ -1,0 +1,109 @@
+"""Prefill/forward parity: CUDA path (through the C ABI) vs the fp64 oracle."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import softmax_learned_covariance_b200 as plx
+from softmax_learned_covariance_b200 import inputs
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def _dev(t16):
+    return t16.torch().to(DEV)
+
+
+def _run_bf16(q, k, v, rho, causal=True, out_dtype=torch.float32):
+    y, lse = plx.parallax_fwd(_dev(q), _dev(k), _dev(v), None if rho is None else _dev(rho), causal=causal,
+                              out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert plx.parallax_last_device_error() == 0
+    return y, lse
+
+
+def test_config1_fp32_tiny_causal():
+    """fp32 path, B=1 H=2 T=128 d=64, rho ~ N(0, 0.1^2); plus the rho = 0 identity."""
+    q, k, v, rho = inputs.fwd_f32_inputs()
+    t = lambda a: torch.from_numpy(a).to(DEV)
+    y, lse = plx.parallax_fwd(t(q), t(k), t(v), t(rho), causal=True)
+    yr, lr = oracle.fwd(q, k, v, rho, causal=True)
+    parity.assert_f32_parity(y.cpu().numpy(), yr, "config1")
+    parity.assert_lse(lse.cpu().numpy(), lr, "config1 lse")
+    y0, _ = plx.parallax_fwd(t(q), t(k), t(v), t(np.zeros_like(rho)), causal=True)
+    yn, _ = plx.parallax_fwd(t(q), t(k), t(v), None, causal=True)
+    assert torch.equal(y0, yn), "rho = 0 must equal the softmax-only instantiation bitwise"
+    ys, _ = oracle.fwd(q, k, v, None, causal=True)
+    parity.assert_f32_parity(y0.cpu().numpy(), ys, "config1 rho=0")
+
+
+@pytest.mark.parametrize("T", [1, 5, 64, 128, 129, 300, 512])
+@pytest.mark.parametrize("causal", [True, False])
+def test_bf16_small_shapes(T, causal):
+    """Several query/key tiles, ragged tails, both masks; rho at the 1.7B-layer scale."""
+    q, k, v, rho = inputs.fwd_bf16_inputs(2, 3, T, 128, seed=100 + T)
+    y, lse = _run_bf16(q, k, v, rho, causal)
+    yr, lr = oracle.fwd(q.f64, k.f64, v.f64, rho.f64, causal=causal)
+    parity.assert_bf16_parity(y.cpu().numpy(), yr, 2, f"T={T} causal={causal}")
+    parity.assert_lse(lse.cpu().numpy(), lr, f"T={T}")
+
+
+def test_bf16_softmax_identity_bitwise():
+    """W_R = 0: the full kernel with rho = 0 equals its softmax-only instantiation bit for bit."""
+    q, k, v, _ = inputs.fwd_bf16_inputs(2, 2, 700, 128, seed=7)
+    zero = inputs.Tensor16(np.zeros_like(q.bits))
+    y0, l0 = _run_bf16(q, k, v, zero)
+    yn, ln = _run_bf16(q, k, v, None)
+    assert torch.equal(y0, yn) and torch.equal(l0, ln)
+    yr, _ = oracle.fwd(q.f64, k.f64, v.f64, None)
+    parity.assert_bf16_parity(yn.cpu().numpy(), yr, 2, "softmax only")
+
+
+def test_bf16_output_dtype():
+    """bf16 y is the rounded fp32 result: within the bf16 gate plus one bf16 ulp of the reference."""
+    q, k, v, rho = inputs.fwd_bf16_inputs(1, 2, 256, 128, seed=9)
+    y32, _ = _run_bf16(q, k, v, rho)
+    y16, _ = _run_bf16(q, k, v, rho, out_dtype=torch.bfloat16)
+    yr, _ = oracle.fwd(q.f64, k.f64, v.f64, rho.f64)
+    ulp = np.abs(inputs.round_bf16(yr)) * 2.0 ** -7
+    err = np.abs(y16.float().cpu().numpy() - yr)
+    assert np.all(err <= parity.BF16_MAX_ABS + ulp)
+    assert torch.equal(y16, y32.to(torch.bfloat16))
+
+
+def test_config3_prefill_1p7b_layer_sampled_rows():
+    """B=8 T=4096 H=16 d=128 (the timed prefill shape): sampled rows of every head vs the oracle."""
+    B, H, T, d = 8, 16, 4096, 128
+    q, k, v, rho = inputs.fwd_bf16_inputs(B, H, T, d, seed=3)
+    y, lse = _run_bf16(q, k, v, rho)
+    y = y.cpu().numpy().reshape(B * H * T, d)
+    lse = lse.cpu().numpy().reshape(-1)
+    base = parity.sample_rows(T, n_head_rows=16, stride=509)
+    heads = np.arange(B * H)
+    rows = (heads[:, None] * T + base[None, :]).reshape(-1)
+    yr, lr = oracle.fwd_rows(q.f64, k.f64, v.f64, rho.f64, rows)
+    parity.assert_bf16_parity(y[rows].reshape(B * H, -1, d), yr.reshape(B * H, -1, d), 1, "config3 rows")
+    parity.assert_lse(lse[rows], lr, "config3 lse")
+
+
+def test_config5_long_context_and_softmax_identity():
+    """B=1 T=32768 H=16: sampled rows vs the oracle, and rho = 0 bitwise equal to softmax only."""
+    B, H, T, d = 1, 16, 32768, 128
+    q, k, v, rho = inputs.fwd_bf16_inputs(B, H, T, d, seed=5)
+    y, lse = _run_bf16(q, k, v, rho)
+    base = np.array(sorted(set(range(8)) | set(range(T - 8, T)) | set(range(0, T, 4099))), np.int64)
+    heads = np.array([0, 7, 15])
+    rows = (heads[:, None] * T + base[None, :]).reshape(-1)
+    yr, lr = oracle.fwd_rows(q.f64, k.f64, v.f64, rho.f64, rows)
+    yg = y.cpu().numpy().reshape(B * H * T, d)[rows]
+    parity.assert_bf16_parity(yg.reshape(len(heads), -1, d), yr.reshape(len(heads), -1, d), 1, "config5 rows")
+    parity.assert_lse(lse.cpu().numpy().reshape(-1)[rows], lr, "config5 lse")
+    del y, lse
+    zero = inputs.Tensor16(np.zeros_like(q.bits))
+    y0, l0 = _run_bf16(q, k, v, zero)
+    yn, ln = _run_bf16(q, k, v, None)
+    assert torch.equal(y0, yn) and torch.equal(l0, ln)
