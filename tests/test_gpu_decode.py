@@ -22,13 +22,13 @@ def _run(q, rho, kc, vc, sl, out_dtype=torch.float32):
     return y, lse
 
 
-def test_config2_decode_step_full():
+def test_decode_b64_h16_ctx4096_all_heads():
     """B=64 H=16 d=128, contiguous cache of 4096 tokens: every head vs the oracle."""
     q, rho, kc, vc, sl = inputs.decode_inputs(64, 16, 4096, 128, seed=2)
     y, lse = _run(q, rho, kc, vc, sl)
     yr, lr = oracle.decode(q.f64, rho.f64, kc.f64, vc.f64, sl)
-    parity.assert_bf16_parity(y.cpu().numpy(), yr, 2, "config2")
-    parity.assert_lse(lse.cpu().numpy(), lr, "config2 lse")
+    parity.assert_bf16_parity(y.cpu().numpy(), yr, 2, "decode b64 ctx4096")
+    parity.assert_lse(lse.cpu().numpy(), lr, "decode b64 ctx4096 lse")
 
 
 @pytest.mark.parametrize("d", [64, 128])

@@ -26,19 +26,19 @@ def _run_bf16(q, k, v, rho, causal=True, out_dtype=torch.float32):
     return y, lse
 
 
-def test_config1_fp32_tiny_causal():
+def test_fp32_tiny_causal_b1_h2_t128_d64():
     """fp32 path, B=1 H=2 T=128 d=64, rho ~ N(0, 0.1^2); plus the rho = 0 identity."""
     q, k, v, rho = inputs.fwd_f32_inputs()
     t = lambda a: torch.from_numpy(a).to(DEV)
     y, lse = plx.parallax_fwd(t(q), t(k), t(v), t(rho), causal=True)
     yr, lr = oracle.fwd(q, k, v, rho, causal=True)
-    parity.assert_f32_parity(y.cpu().numpy(), yr, "config1")
-    parity.assert_lse(lse.cpu().numpy(), lr, "config1 lse")
+    parity.assert_f32_parity(y.cpu().numpy(), yr, "fp32 tiny")
+    parity.assert_lse(lse.cpu().numpy(), lr, "fp32 tiny lse")
     y0, _ = plx.parallax_fwd(t(q), t(k), t(v), t(np.zeros_like(rho)), causal=True)
     yn, _ = plx.parallax_fwd(t(q), t(k), t(v), None, causal=True)
     assert torch.equal(y0, yn), "rho = 0 must equal the softmax-only instantiation bitwise"
     ys, _ = oracle.fwd(q, k, v, None, causal=True)
-    parity.assert_f32_parity(y0.cpu().numpy(), ys, "config1 rho=0")
+    parity.assert_f32_parity(y0.cpu().numpy(), ys, "fp32 tiny rho=0")
 
 
 @pytest.mark.parametrize("T", [1, 5, 64, 128, 129, 300, 512])
@@ -75,7 +75,7 @@ def test_bf16_output_dtype():
     assert torch.equal(y16, y32.to(torch.bfloat16))
 
 
-def test_config3_prefill_1p7b_layer_sampled_rows():
+def test_prefill_b8_t4096_h16_sampled_rows():
     """B=8 T=4096 H=16 d=128 (the timed prefill shape): sampled rows of every head vs the oracle."""
     B, H, T, d = 8, 16, 4096, 128
     q, k, v, rho = inputs.fwd_bf16_inputs(B, H, T, d, seed=3)
@@ -86,11 +86,11 @@ def test_config3_prefill_1p7b_layer_sampled_rows():
     heads = np.arange(B * H)
     rows = (heads[:, None] * T + base[None, :]).reshape(-1)
     yr, lr = oracle.fwd_rows(q.f64, k.f64, v.f64, rho.f64, rows)
-    parity.assert_bf16_parity(y[rows].reshape(B * H, -1, d), yr.reshape(B * H, -1, d), 1, "config3 rows")
-    parity.assert_lse(lse[rows], lr, "config3 lse")
+    parity.assert_bf16_parity(y[rows].reshape(B * H, -1, d), yr.reshape(B * H, -1, d), 1, "prefill b8 t4096 rows")
+    parity.assert_lse(lse[rows], lr, "prefill b8 t4096 lse")
 
 
-def test_config5_long_context_and_softmax_identity():
+def test_long_prefill_t32768_and_softmax_identity():
     """B=1 T=32768 H=16: sampled rows vs the oracle, and rho = 0 bitwise equal to softmax only."""
     B, H, T, d = 1, 16, 32768, 128
     q, k, v, rho = inputs.fwd_bf16_inputs(B, H, T, d, seed=5)
@@ -100,8 +100,8 @@ def test_config5_long_context_and_softmax_identity():
     rows = (heads[:, None] * T + base[None, :]).reshape(-1)
     yr, lr = oracle.fwd_rows(q.f64, k.f64, v.f64, rho.f64, rows)
     yg = y.cpu().numpy().reshape(B * H * T, d)[rows]
-    parity.assert_bf16_parity(yg.reshape(len(heads), -1, d), yr.reshape(len(heads), -1, d), 1, "config5 rows")
-    parity.assert_lse(lse.cpu().numpy().reshape(-1)[rows], lr, "config5 lse")
+    parity.assert_bf16_parity(yg.reshape(len(heads), -1, d), yr.reshape(len(heads), -1, d), 1, "t32768 rows")
+    parity.assert_lse(lse.cpu().numpy().reshape(-1)[rows], lr, "t32768 lse")
     del y, lse
     zero = inputs.Tensor16(np.zeros_like(q.bits))
     y0, l0 = _run_bf16(q, k, v, zero)

@@ -31,7 +31,7 @@ def test_small_shapes_full(B, T, dm, H, d):
     _check_rho(rho.float().cpu().numpy(), ref, f"{(B, T, dm, H, d)}")
 
 
-def test_config3_projection_sampled_tokens_and_pipeline():
+def test_projection_b8_t4096_dm2048_and_pipeline():
     """x [8,4096,2048], W_R [2048, 16*128]: sampled token rows vs the oracle; then rho_proj -> fwd
     on sampled rows vs the oracle run on the bf16-stored probe."""
     B, T, dm, H, d = 8, 4096, 2048, 16, 128
@@ -42,7 +42,7 @@ def test_config3_projection_sampled_tokens_and_pipeline():
     ref = oracle.rho_proj(x.f64, w.f64, H, d, bt_list=bt)          # [n, H, d]
     g = rho.float().cpu().numpy()                                     # [B, H, T, d]
     gs = g[bt // T, :, bt % T, :]
-    _check_rho(gs, ref, "config3 rho")
+    _check_rho(gs, ref, "rho b8 t4096")
 
     q, k, v, _ = inputs.fwd_bf16_inputs(B, H, T, d, seed=33)
     y, _ = plx.parallax_fwd(q.torch().to(DEV), k.torch().to(DEV), v.torch().to(DEV), rho)
