@@ -123,6 +123,51 @@ class ClockSampler:
 # --------------------------------------------------------------------------- #
 # our arm
 # --------------------------------------------------------------------------- #
+def run_profile_case(args):
+    """Small single-kernel loops for ncu captures (inputs still larger than L2, a few GB at most).
+
+    profile_fwd    : parallax_fwd, B=2 H=16 T=8192 d=128 causal (plus its rho input)
+    profile_decode : parallax_decode, B=16 H=16 d=128, 8192-token cache
+    profile_rho    : parallax_rho_proj, x [2, 8192, 2048] @ W_R [2048, 2048]
+    """
+    import torch
+
+    import softmax_learned_covariance_b200 as plx
+    from softmax_learned_covariance_b200 import inputs
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    if args.workload == "profile_fwd":
+        q, k, v, r = (t.torch().to(dev) for t in inputs.fwd_bf16_inputs(2, 16, 8192, 128, seed=3))
+        y = torch.empty(q.shape, dtype=torch.float32, device=dev)
+        call = lambda: plx.parallax_fwd(q, k, v, r, y=y, want_lse=False)
+        work, unit = prefill_flops(2, 16, 8192, 128), "TFLOP/s"
+    elif args.workload == "profile_decode":
+        q, r, kc, vc, sl = inputs.decode_inputs(16, 16, 8192, 128, seed=2)
+        q, r, kc, vc = (t.torch().to(dev) for t in (q, r, kc, vc))
+        dsl = torch.from_numpy(sl).to(dev)
+        y = torch.empty((16, 16, 128), dtype=torch.float32, device=dev)
+        call = lambda: plx.parallax_decode(q, r, kc, vc, dsl, y=y, want_lse=False)
+        work, unit = decode_bytes(16, 16, 128, sl), "TB/s"
+    else:
+        x, w = (t.torch().to(dev) for t in inputs.rho_proj_inputs(2, 8192, 2048, 16, 128, seed=3))
+        r = torch.empty((2, 16, 8192, 128), dtype=torch.bfloat16, device=dev)
+        call = lambda: plx.parallax_rho_proj(x, w, 16, 128, rho=r)
+        work, unit = rho_proj_flops(2, 8192, 2048, 16, 128), "TFLOP/s"
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        call()
+    b.record()
+    torch.cuda.synchronize()
+    assert plx.parallax_last_device_error() == 0
+    ms = a.elapsed_time(b) / args.steps
+    return {"workload": args.workload, "ms": ms, "value": work / (ms * 1e-3) / 1e12, "unit": unit}
+
+
 def run_ours(args, rank, world):
     import torch
 
@@ -345,7 +390,8 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["default", "prefill_long"], default="default")
+    ap.add_argument("--workload", choices=["default", "prefill_long", "profile_fwd", "profile_decode",
+                                           "profile_rho"], default="default")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -363,6 +409,9 @@ def main():
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
 
+    if args.workload.startswith("profile_"):
+        print(json.dumps(run_profile_case(args)), flush=True)
+        return
     if args.impl == "reference":
         line = run_reference(args, rank, world)
     else:
