@@ -129,6 +129,34 @@ PARALLAX_API int parallax_decode_ex(const void *q, const void *rho, const void *
                        parallax_stream_t stream);
 
 /*
+ * parallax_decode_noalloc -- parallax_decode that never allocates device memory.
+ *
+ * The pages have no counterpart to this call.  It is for callers that must not
+ * have a library allocate on their behalf: serving engines that reserve the
+ * device's memory through their own pool at start-up and run under a fixed
+ * budget, decode loops where a cudaMalloc, or the device-wide synchronization
+ * of a cudaFree, would stall every stream, and plugin interfaces whose execute
+ * callbacks forbid allocation.
+ *
+ * Same arguments, results and errors as parallax_decode.  The split partials
+ * live in a static device array of PARALLAX_DECODE_NOALLOC_SCRATCH_BYTES
+ * (16 MiB) compiled into the library; every GPU that loads the library holds
+ * it until the process exits.  A shape whose partials need more than that
+ * (parallax_decode_workspace_bytes tells) returns PARALLAX_ERR_SHAPE and
+ * enqueues nothing.  The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress) with that device current; make that first
+ * call before any stream capture.  All calls on a device share the array and
+ * it keeps the last call's contents (nothing in it needs clearing between
+ * calls), so calls that overlap on the GPU, e.g. on two streams at once, race:
+ * the caller must serialize them.
+ */
+#define PARALLAX_DECODE_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+PARALLAX_API int parallax_decode_noalloc(const void *q, const void *rho, const void *kcache,
+                                         const void *vcache, const int *seqlens, void *y, float *lse,
+                                         int B, int H, int Tcap, int d, int in_dtype, int out_dtype,
+                                         parallax_stream_t stream);
+
+/*
  * parallax_rho_proj -- the learned probe rho = x W_R, split per head.
  *
  * Passage: encorp.ai blog, section "Por que eliminar el solucionador de
