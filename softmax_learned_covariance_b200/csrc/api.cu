@@ -24,7 +24,8 @@ constexpr int MAX_DEVICES = 64;
 struct DevState {
     bool init = false;
     int sms = 0;
-    int *err = nullptr;
+    int *err = nullptr;           // device error word (ctl[0])
+    int *counter = nullptr;       // persistent-grid work counter (ctl[32])
     void *ws = nullptr;
     size_t ws_bytes = 0;
 };
@@ -42,8 +43,9 @@ int get_state(DevState **out) {
     DevState &s = g_dev[dev];
     if (!s.init) {
         if (cudaDeviceGetAttribute(&s.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return PARALLAX_ERR_CUDA;
-        if (cudaMalloc(&s.err, sizeof(int)) != cudaSuccess) return PARALLAX_ERR_CUDA;
-        if (cudaMemset(s.err, 0, sizeof(int)) != cudaSuccess) return PARALLAX_ERR_CUDA;
+        if (cudaMalloc(&s.err, 256) != cudaSuccess) return PARALLAX_ERR_CUDA;
+        if (cudaMemset(s.err, 0, 256) != cudaSuccess) return PARALLAX_ERR_CUDA;
+        s.counter = s.err + 32;
         s.init = true;
     }
     *out = &s;
@@ -72,9 +74,11 @@ int get_workspace(DevState *s, size_t bytes, void **out) {
     return PARALLAX_OK;
 }
 
-DeviceCtl make_ctl(const DevState *s) {
+}  // namespace
+
+DeviceCtl plx::ctl_from_env(int *err) {
     DeviceCtl c;
-    c.err = s->err;
+    c.err = err;
     unsigned long long ms = 2000;
     if (const char *e = std::getenv("PARALLAX_WAIT_TIMEOUT_MS")) {
         const long v = std::strtol(e, nullptr, 10);
@@ -85,6 +89,10 @@ DeviceCtl make_ctl(const DevState *s) {
     if (const char *e = std::getenv("PARALLAX_DEBUG_FLAGS")) c.debug_flags = (unsigned)std::strtoul(e, nullptr, 0);
     return c;
 }
+
+namespace {
+
+DeviceCtl make_ctl(const DevState *s) { return ctl_from_env(s->err); }
 
 int ensure_encoder() {
     std::lock_guard<std::mutex> lk(g_mu);
@@ -151,6 +159,12 @@ int parallax_last_device_error(parallax_stream_t stream) {
     int v = 0;
     if (cudaMemcpy(&v, s->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return PARALLAX_ERR_CUDA;
     if (v != 0 && cudaMemset(s->err, 0, sizeof(int)) != cudaSuccess) return PARALLAX_ERR_CUDA;
+    if (int *w = noalloc_error_word()) {
+        int v2 = 0;
+        if (cudaMemcpy(&v2, w, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return PARALLAX_ERR_CUDA;
+        if (v2 != 0 && cudaMemset(w, 0, sizeof(int)) != cudaSuccess) return PARALLAX_ERR_CUDA;
+        if (v == 0) v = v2;
+    }
     return v;
 }
 
@@ -192,7 +206,7 @@ int parallax_fwd(const void *q, const void *k, const void *v, const void *rho, v
         tm.r = tm.q;
     }
     return status_of(
-        launch_fwd_sm100(tm, rho != nullptr, y, lse, B, H, T, d, causal, out_dtype, s->sms, make_ctl(s), cs));
+        launch_fwd_sm100(tm, rho != nullptr, y, lse, B, H, T, d, causal, out_dtype, s->sms, s->counter, make_ctl(s), cs));
 }
 
 size_t parallax_decode_workspace_bytes(int B, int H, int Tcap, int d) {
@@ -228,7 +242,7 @@ static int decode_impl(const void *q, const void *rho, const void *kcache, const
         ws = workspace;
     }
     return status_of(launch_decode(q, rho, kcache, vcache, seqlens, y, lse, B, H, Tcap, d, out_dtype, plan,
-                                   static_cast<float *>(ws), static_cast<cudaStream_t>(stream)));
+                                   static_cast<float *>(ws), s->sms, make_ctl(s), static_cast<cudaStream_t>(stream)));
 }
 
 int parallax_decode(const void *q, const void *rho, const void *kcache, const void *vcache, const int *seqlens,

@@ -28,10 +28,14 @@ constexpr int kMaxDevices = 64;
 
 // Shared by every call on a device; keeps the last call's contents.
 static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
+// Where this entry point's kernels record a bounded wait that gave up
+// (read and cleared by parallax_last_device_error).
+static __device__ int g_noalloc_err;
 
 struct NoallocDevice {
     bool ready = false;
     void *scratch = nullptr;   // device address of g_decode_scratch on this device
+    int *err = nullptr;        // device address of g_noalloc_err on this device
     int sms = 0;
 };
 std::mutex g_noalloc_mu;
@@ -42,18 +46,31 @@ int noalloc_setup(int dev, NoallocDevice **out) {
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
     NoallocDevice &s = g_noalloc_dev[dev];
     if (!s.ready) {
-        void *p = nullptr;
+        void *p = nullptr, *e = nullptr;
         if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return PARALLAX_ERR_CUDA;
+        if (cudaGetSymbolAddress(&e, g_noalloc_err) != cudaSuccess || e == nullptr) return PARALLAX_ERR_CUDA;
         int sms = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
             return PARALLAX_ERR_CUDA;
         s.scratch = p;
+        s.err = static_cast<int *>(e);
         s.sms = sms;
         s.ready = true;
     }
     *out = &s;
     return PARALLAX_OK;
 }
+
+}  // namespace
+
+int *plx::noalloc_error_word() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    return g_noalloc_dev[dev].ready ? g_noalloc_dev[dev].err : nullptr;
+}
+
+namespace {
 
 bool is_aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
@@ -82,6 +99,7 @@ extern "C" PARALLAX_API int parallax_decode_noalloc(const void *q, const void *r
     // so nothing in the array has to be cleared between calls.
     if (plx::decode_partials_bytes(B, H, d, plan) > kScratchBytes) return PARALLAX_ERR_SHAPE;
     const cudaError_t e = plx::launch_decode(q, rho, kcache, vcache, seqlens, y, lse, B, H, Tcap, d, out_dtype, plan,
-                                             static_cast<float *>(s->scratch), static_cast<cudaStream_t>(stream));
+                                             static_cast<float *>(s->scratch), s->sms, plx::ctl_from_env(s->err),
+                                             static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PARALLAX_OK : PARALLAX_ERR_CUDA;
 }

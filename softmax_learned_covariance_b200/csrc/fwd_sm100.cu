@@ -19,11 +19,13 @@
 // rescales (the running max is only moved when it rises by more than 8 in
 // log2 units; O and M are then rescaled in TMEM).
 //
-// Roles (256 threads, one CTA per SM, persistent over (head, query tile)
-// items in longest-first order):
-//   warp 0      TMA producer: Q and R per item, K and V(fp16) rings per key tile
+// Roles (384 threads, one CTA per SM, persistent over (head, query tile)
+// items taken longest-first from an atomic work counter):
+//   warp 0      scheduler + TMA producer: Q and R per item, K and V(fp16) rings
 //   warp 1      TMEM owner and single-thread UMMA issuer
-//   warps 4..7  softmax/correction and epilogue, one query row per thread
+//   warps 4..11 two softmax warpgroups, one query row per thread in each; the
+//               group g handles key columns [32g, 32g+32) of every 64-key tile,
+//               the two exchange their partial row max through shared memory
 // TMEM (512 columns): O [0,128) | M' [128,256) | S0 | A0 | S1 | A1 (64 each),
 // S/A double-buffered so the score UMMAs of tile j+1 run while tile j is
 // exponentiated.
@@ -45,9 +47,12 @@ namespace {
 constexpr int D = 128;
 constexpr int BM = 128;          // query rows per tile
 constexpr int BN = 64;           // keys per tile
+constexpr int HALF = BN / 2;     // key columns per softmax warpgroup
 constexpr int KST = 4;           // K ring stages
 constexpr int VST = 4;           // V ring stages
-constexpr int NTHREADS = 256;
+constexpr int SCHED = 4;         // scheduler ring depth (items in flight)
+constexpr int NTHREADS = 384;
+constexpr int NSOFT = 256;       // softmax threads (two warpgroups)
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 constexpr float RESCALE_THRESHOLD = 8.0f;   // log2 units
@@ -62,6 +67,9 @@ constexpr int V_BYTES = BN * D * 2;    // 16 KB fp16, two d-halves of [64 keys x
 constexpr uint32_t COL_O = 0, COL_M = 128;
 __host__ __device__ constexpr uint32_t col_s(uint32_t b) { return 256 + b * 128; }
 __host__ __device__ constexpr uint32_t col_a(uint32_t b) { return 256 + b * 128 + 64; }
+// fp16 P (or P o A') of key group kk (16 keys) inside the S (or A) buffer: each
+// warpgroup packs its 32 keys into the first 16 columns of its own 32-column half.
+__host__ __device__ constexpr uint32_t col_p16(uint32_t kk) { return (kk >> 1) * 32 + (kk & 1) * 8; }
 
 constexpr uint32_t IDESC_S = idesc_f16(1, 1, 0, 0, BM, BN);     // bf16 Q/R (K-major) x bf16 K (K-major)
 constexpr uint32_t IDESC_PV = idesc_f16(0, 0, 0, 1, BM, D);     // f16 P (TMEM) x f16 V (MN-major)
@@ -72,8 +80,14 @@ struct __align__(8) Bars {
     uint64_t v_full[VST], v_empty[VST];
     uint64_t s_full[2], p_full[2], pv_done[2];
     uint64_t om_free;
+    uint64_t sched_full[SCHED], sched_empty[SCHED];
+    uint64_t xchg[2];            // per tile parity: both softmax groups posted their partial max
+    uint64_t esum;               // per item: both softmax groups posted their partial sums
+    int sched_item[SCHED];
     uint32_t tmem_base;
     int abort_flag;
+    float red_max[2][2][BM];     // [tile parity][warpgroup][row] partial row max
+    float red_sum[2][2][BM];     // [l or abar'][warpgroup][row] partial sums for the epilogue
 };
 
 constexpr size_t SMEM_BYTES = 1024 + 2 * (size_t)Q_BYTES + (size_t)KST * K_BYTES + (size_t)VST * V_BYTES + sizeof(Bars);
@@ -91,11 +105,33 @@ __device__ __forceinline__ Item item_of(int w, int BH, int nq, int T, int causal
     return it;
 }
 
+// Bounded wait whose outcome is the same for all 32 lanes (lanes that saw the
+// phase complete still give up if another lane of the warp gave up), so the
+// .sync.aligned tcgen05 instructions that follow are never reached divergently.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const WaitCtl &wc) {
+    const bool got = mbar_wait(bar, parity, wc);
+    return __all_sync(0xffffffffu, got);
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// Consumers take the k-th scheduled item from the ring (same sequence in every role).
+__device__ __forceinline__ bool next_item(Bars *bars, uint32_t k, int &w, const WaitCtl &wc) {
+    const uint32_t s = k % SCHED;
+    if (!mbar_wait(smem_u32(&bars->sched_full[s]), (k / SCHED) & 1, wc)) return false;
+    w = bars->sched_item[s];
+    return true;
+}
+
 template <bool WITH_RHO, typename Tout>
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
           const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_v, Tout *__restrict__ y,
-          float *__restrict__ lse, int BH, int T, int causal, DeviceCtl ctl) {
+          float *__restrict__ lse, int BH, int T, int causal, int *__restrict__ work_counter, DeviceCtl ctl) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sQ = smem;
@@ -118,10 +154,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&bars->s_full[b]), 1);
-            mbar_init(smem_u32(&bars->p_full[b]), 128);
+            mbar_init(smem_u32(&bars->p_full[b]), NSOFT);
             mbar_init(smem_u32(&bars->pv_done[b]), 1);
         }
-        mbar_init(smem_u32(&bars->om_free), 128);
+        mbar_init(smem_u32(&bars->om_free), NSOFT);
+        for (int s = 0; s < SCHED; ++s) {
+            mbar_init(smem_u32(&bars->sched_full[s]), 1);
+            mbar_init(smem_u32(&bars->sched_empty[s]), 1 + NSOFT / 32);   // UMMA thread + one lane per softmax warp
+        }
+        mbar_init(smem_u32(&bars->xchg[0]), NSOFT);
+        mbar_init(smem_u32(&bars->xchg[1]), NSOFT);
+        mbar_init(smem_u32(&bars->esum), NSOFT);
         bars->abort_flag = 0;
         fence_mbar_init();
     }
@@ -139,14 +182,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int items = nq * BH;
 
     if (warp == 0 && lane == 0) {
-        // ======================================================= producer ==
+        // ============================================= scheduler + producer ==
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
         if (WITH_RHO) tma_prefetch_desc(&tm_r);
-        uint32_t kc = 0, vc = 0, ic = 0;
+        uint32_t kc = 0, vc = 0;
         bool ok = true;
-        for (int w = blockIdx.x; w < items && ok; w += gridDim.x, ++ic) {
+        for (uint32_t ic = 0; ok; ++ic) {
+            const uint32_t ss = ic % SCHED;
+            if (!mbar_wait(smem_u32(&bars->sched_empty[ss]), ((ic / SCHED) & 1) ^ 1, wc)) break;
+            const int w = ic == 0 ? (int)blockIdx.x : (int)gridDim.x + atomicAdd(work_counter, 1);
+            bars->sched_item[ss] = w;
+            mbar_arrive(smem_u32(&bars->sched_full[ss]));
+            if (w >= items) break;
             const Item it = item_of(w, BH, nq, T, causal);
             const int q0 = it.qt * BM;
             if (!mbar_wait(smem_u32(&bars->qr_empty), (ic & 1) ^ 1, wc)) break;
@@ -186,7 +235,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
     } else if (warp == 1 && lane == 0) {
         // ==================================================== UMMA issuer ==
-        uint32_t kc = 0, vc = 0, ic = 0, G = 0;
+        uint32_t kc = 0, vc = 0, G = 0;
         bool ok = true;
         const uint32_t q_base = smem_u32(sQ), r_base = smem_u32(sR);
         auto issue_pv = [&](uint32_t g, bool first, uint32_t icur) -> bool {
@@ -202,15 +251,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             for (int kk = 0; kk < BN / 16; ++kk) {
                 const uint64_t vdesc = sdesc_sw128(vb + kk * 16 * 128, V_BYTES / 2, 1024);
                 const uint32_t acc = (!first || kk > 0) ? 1u : 0u;
-                umma_ts(tmem + COL_O, tmem + col_s(b) + kk * 8, vdesc, IDESC_PV, acc);
-                if constexpr (WITH_RHO) umma_ts(tmem + COL_M, tmem + col_a(b) + kk * 8, vdesc, IDESC_PV, acc);
+                umma_ts(tmem + COL_O, tmem + col_s(b) + col_p16(kk), vdesc, IDESC_PV, acc);
+                if constexpr (WITH_RHO) umma_ts(tmem + COL_M, tmem + col_a(b) + col_p16(kk), vdesc, IDESC_PV, acc);
             }
             tc_commit(smem_u32(&bars->v_empty[s]));
             tc_commit(smem_u32(&bars->pv_done[b]));
             ++vc;
             return true;
         };
-        for (int w = blockIdx.x; w < items && ok; w += gridDim.x, ++ic) {
+        for (uint32_t ic = 0; ok; ++ic) {
+            int w;
+            if (!next_item(bars, ic, w, wc)) break;
+            mbar_arrive(smem_u32(&bars->sched_empty[ic % SCHED]));
+            if (w >= items) break;
             const Item it = item_of(w, BH, nq, T, causal);
             if (!mbar_wait(smem_u32(&bars->qr_full), ic & 1, wc)) break;
             for (int j = 0; j < it.nkv; ++j, ++G) {
@@ -241,61 +294,81 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
     } else if (warp >= 4) {
         // ============================================ softmax + epilogue ==
+        const int grp = (warp - 4) >> 2;                 // 0: key columns [0,32), 1: [32,64)
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;               // query row within the tile == TMEM lane
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const float scale_log2 = LOG2E / sqrtf((float)D);
-        uint32_t G = 0, ic = 0;
+        uint32_t G = 0, ni = 0;   // key tiles and items processed by this CTA
         bool ok = true;
-        for (int w = blockIdx.x; w < items && ok; w += gridDim.x, ++ic) {
+        for (uint32_t ic = 0; ok; ++ic) {
+            int w = 0;
+            const bool got = next_item(bars, ic, w, wc);
+            if (!__all_sync(0xffffffffu, got)) break;
+            if (lane == 0) mbar_arrive(smem_u32(&bars->sched_empty[ic % SCHED]));
+            if (w >= items) break;
             const Item it = item_of(w, BH, nq, T, causal);
             const int qrow = it.qt * BM + r;
-            float m_ref = -INFINITY, l = 0.f, ab = 0.f;
+            const int kvis = causal ? min(T, qrow + 1) : T;  // keys visible to this row
+            float m_ref = -INFINITY;
+            float l4[4] = {0.f, 0.f, 0.f, 0.f}, a4[4] = {0.f, 0.f, 0.f, 0.f};
             for (int j = 0; j < it.nkv; ++j, ++G) {
                 const uint32_t b = G & 1;
-                if (!mbar_wait(smem_u32(&bars->s_full[b]), (G >> 1) & 1, wc)) { ok = false; break; }
+                if (!warp_wait(smem_u32(&bars->s_full[b]), (G >> 1) & 1, wc)) { ok = false; break; }
                 tc_fence_after();
-                uint32_t sr[BN];
-                uint32_t ar[WITH_RHO ? BN : 1];
-#pragma unroll
-                for (int c = 0; c < BN; c += 16) {
-                    tmem_ld16(tmem + lane_off + col_s(b) + c, *reinterpret_cast<uint32_t(*)[16]>(&sr[c]));
-                    if constexpr (WITH_RHO)
-                        tmem_ld16(tmem + lane_off + col_a(b) + c, *reinterpret_cast<uint32_t(*)[16]>(&ar[c]));
+                uint32_t sr[HALF];
+                uint32_t ar[WITH_RHO ? HALF : 1];
+                tmem_ld16(tmem + lane_off + col_s(b) + grp * HALF, *reinterpret_cast<uint32_t(*)[16]>(&sr[0]));
+                tmem_ld16(tmem + lane_off + col_s(b) + grp * HALF + 16, *reinterpret_cast<uint32_t(*)[16]>(&sr[16]));
+                if constexpr (WITH_RHO) {
+                    tmem_ld16(tmem + lane_off + col_a(b) + grp * HALF, *reinterpret_cast<uint32_t(*)[16]>(&ar[0]));
+                    tmem_ld16(tmem + lane_off + col_a(b) + grp * HALF + 16,
+                              *reinterpret_cast<uint32_t(*)[16]>(&ar[16]));
                 }
                 tmem_wait_ld();
-                // visible keys of this row in this tile: c < limit
-                const int k0 = j * BN;
-                int limit = (causal ? min(T, qrow + 1) : T) - k0;
-                float mx = -INFINITY;
-                if (limit >= BN) {
+                // keys of this tile visible to this row: c < limit
+                const int limit = kvis - (j * BN + grp * HALF);
+                if (limit < HALF) {
 #pragma unroll
-                    for (int c = 0; c < BN; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
-                } else {
-#pragma unroll
-                    for (int c = 0; c < BN; ++c) {
+                    for (int c = 0; c < HALF; ++c)
                         if (c >= limit) sr[c] = __float_as_uint(-INFINITY);
-                        mx = fmaxf(mx, __uint_as_float(sr[c]));
-                    }
                 }
-                mx *= scale_log2;
+                float mx;
+                {
+                    float t[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        t[i] = fmax3(__uint_as_float(sr[i]), __uint_as_float(sr[i + 8]),
+                                     __uint_as_float(sr[i + 16]));
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) t[i] = fmaxf(t[i], __uint_as_float(sr[i + 24]));
+                    mx = fmaxf(fmax3(t[0], t[1], t[2]), fmax3(t[3], t[4], fmax3(t[5], t[6], t[7])));
+                }
+                bars->red_max[G & 1][grp][r] = mx;
+                mbar_arrive(smem_u32(&bars->xchg[G & 1]));
+                if (!warp_wait(smem_u32(&bars->xchg[G & 1]), (G >> 1) & 1, wc)) { ok = false; break; }
+                mx = fmaxf(mx, bars->red_max[G & 1][grp ^ 1][r]) * scale_log2;
                 float alpha = 1.f;
                 bool moved = false;
                 if (mx > m_ref + RESCALE_THRESHOLD) {
                     alpha = ex2(m_ref - mx);     // 0 when m_ref = -inf
                     m_ref = mx;
-                    l *= alpha;
-                    ab *= alpha;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        l4[i] *= alpha;
+                        a4[i] *= alpha;
+                    }
                     moved = true;
                 }
-                // O and M' hold earlier tiles of this item: rescale them in TMEM.
+                // O and M' hold earlier tiles of this item: rescale them in TMEM,
+                // each warpgroup its half of the columns.
                 if (__any_sync(0xffffffffu, moved && j > 0)) {
                     const uint32_t gp = G - 1;
-                    if (!mbar_wait(smem_u32(&bars->pv_done[gp & 1]), (gp >> 1) & 1, wc)) { ok = false; break; }
+                    if (!warp_wait(smem_u32(&bars->pv_done[gp & 1]), (gp >> 1) & 1, wc)) { ok = false; break; }
                     tc_fence_after();
                     const float f = (moved && j > 0) ? alpha : 1.f;
 #pragma unroll 1
-                    for (int c = 0; c < D; c += 16) {
+                    for (int c = grp * 64; c < grp * 64 + 64; c += 16) {
                         uint32_t t[16];
                         tmem_ld16(tmem + lane_off + COL_O + c, t);
                         tmem_wait_ld();
@@ -311,48 +384,51 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         }
                     }
                 }
-                // P = exp2(z*log2e - m_ref) as fp16, P o A' as fp16, sums from the rounded values
+                // P = exp2(z*log2e - m_ref) as fp16; P o A' as fp16; sums from the rounded values
                 const float neg_m = -m_ref;
-                uint32_t pk[BN / 2];
-                uint32_t pak[WITH_RHO ? BN / 2 : 1];
+                uint32_t pk[HALF / 2];
+                uint32_t pak[WITH_RHO ? HALF / 2 : 1];
 #pragma unroll
-                for (int i = 0; i < BN / 2; ++i) {
+                for (int i = 0; i < HALF / 2; ++i) {
                     const float p0 = ex2(fmaf(__uint_as_float(sr[2 * i]), scale_log2, neg_m));
                     const float p1 = ex2(fmaf(__uint_as_float(sr[2 * i + 1]), scale_log2, neg_m));
                     pk[i] = pack_f16x2(p0, p1);
-                    l = add_f16x2_to_f32(l, pk[i]);
+                    l4[i & 3] = add_f16x2_to_f32(l4[i & 3], pk[i]);
                     if constexpr (WITH_RHO) {
                         const uint32_t ah = pack_f16x2(__uint_as_float(ar[2 * i]) * A_SCALE,
                                                        __uint_as_float(ar[2 * i + 1]) * A_SCALE);
                         pak[i] = hmul2(pk[i], ah);
-                        ab = add_f16x2_to_f32(ab, pak[i]);
+                        a4[i & 3] = add_f16x2_to_f32(a4[i & 3], pak[i]);
                     }
                 }
-                tmem_st16(tmem + lane_off + col_s(b), *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
-                tmem_st16(tmem + lane_off + col_s(b) + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
-                if constexpr (WITH_RHO) {
-                    tmem_st16(tmem + lane_off + col_a(b), *reinterpret_cast<uint32_t(*)[16]>(&pak[0]));
-                    tmem_st16(tmem + lane_off + col_a(b) + 16, *reinterpret_cast<uint32_t(*)[16]>(&pak[16]));
-                }
+                tmem_st16(tmem + lane_off + col_s(b) + grp * HALF, pk);
+                if constexpr (WITH_RHO) tmem_st16(tmem + lane_off + col_a(b) + grp * HALF, pak);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(smem_u32(&bars->p_full[b]));
             }
             if (!ok) break;
             // ---------------------------------------------- epilogue --
+            bars->red_sum[0][grp][r] = (l4[0] + l4[1]) + (l4[2] + l4[3]);
+            bars->red_sum[1][grp][r] = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+            mbar_arrive(smem_u32(&bars->esum));
+            if (!warp_wait(smem_u32(&bars->esum), ni & 1, wc)) break;
+            ++ni;
+            const float l = bars->red_sum[0][0][r] + bars->red_sum[0][1][r];
+            const float ab = bars->red_sum[1][0][r] + bars->red_sum[1][1][r];
             const uint32_t glast = G - 1;
             if (it.nkv >= 2) {
                 const uint32_t gp = glast - 1;
-                if (!mbar_wait(smem_u32(&bars->pv_done[gp & 1]), (gp >> 1) & 1, wc)) break;
+                if (!warp_wait(smem_u32(&bars->pv_done[gp & 1]), (gp >> 1) & 1, wc)) break;
             }
-            if (!mbar_wait(smem_u32(&bars->pv_done[glast & 1]), (glast >> 1) & 1, wc)) break;
+            if (!warp_wait(smem_u32(&bars->pv_done[glast & 1]), (glast >> 1) & 1, wc)) break;
             tc_fence_after();
             const float inv_l = 1.0f / l;
             const float abar = ab * inv_l;
             const bool store = qrow < T;
             Tout *yrow = y + ((size_t)it.bh * T + (store ? qrow : 0)) * D;
 #pragma unroll 1
-            for (int c = 0; c < D; c += 16) {
+            for (int c = grp * 64; c < grp * 64 + 64; c += 16) {
                 uint32_t o[16], mm[16];
                 tmem_ld16(tmem + lane_off + COL_O + c, o);
                 if constexpr (WITH_RHO) tmem_ld16(tmem + lane_off + COL_M + c, mm);
@@ -387,7 +463,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     }
                 }
             }
-            if (store && lse != nullptr) lse[(size_t)it.bh * T + qrow] = (m_ref + log2f(l)) * LN2;
+            if (store && grp == 0 && lse != nullptr) lse[(size_t)it.bh * T + qrow] = (m_ref + log2f(l)) * LN2;
             tc_fence_before();
             mbar_arrive(smem_u32(&bars->om_free));
         }
@@ -403,7 +479,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
 template <bool WITH_RHO, typename Tout>
 cudaError_t launch_t(const FwdTensorMaps &tm, void *y, float *lse, int BH, int T, int causal, int sm_count,
-                     const DeviceCtl &ctl, cudaStream_t s) {
+                     int *work_counter, const DeviceCtl &ctl, cudaStream_t s) {
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(k_fwd<WITH_RHO, Tout>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -413,23 +489,26 @@ cudaError_t launch_t(const FwdTensorMaps &tm, void *y, float *lse, int BH, int T
     }
     const int items = ((T + BM - 1) / BM) * BH;
     const int grid = items < sm_count ? items : sm_count;
+    cudaError_t e = cudaMemsetAsync(work_counter, 0, sizeof(int), s);
+    if (e != cudaSuccess) return e;
     k_fwd<WITH_RHO, Tout><<<grid, NTHREADS, SMEM_BYTES, s>>>(tm.q, tm.k, tm.r, tm.v16, static_cast<Tout *>(y), lse,
-                                                             BH, T, causal, ctl);
+                                                             BH, T, causal, work_counter, ctl);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_fwd_sm100(const FwdTensorMaps &tm, bool with_rho, void *y, float *lse, int B, int H, int T,
-                             int d, int causal, int out_dtype, int sm_count, const DeviceCtl &ctl, cudaStream_t s) {
+                             int d, int causal, int out_dtype, int sm_count, int *work_counter, const DeviceCtl &ctl,
+                             cudaStream_t s) {
     (void)d;
     const int BH = B * H;
     if (out_dtype == PARALLAX_F32) {
-        if (with_rho) return launch_t<true, float>(tm, y, lse, BH, T, causal, sm_count, ctl, s);
-        return launch_t<false, float>(tm, y, lse, BH, T, causal, sm_count, ctl, s);
+        if (with_rho) return launch_t<true, float>(tm, y, lse, BH, T, causal, sm_count, work_counter, ctl, s);
+        return launch_t<false, float>(tm, y, lse, BH, T, causal, sm_count, work_counter, ctl, s);
     }
-    if (with_rho) return launch_t<true, __nv_bfloat16>(tm, y, lse, BH, T, causal, sm_count, ctl, s);
-    return launch_t<false, __nv_bfloat16>(tm, y, lse, BH, T, causal, sm_count, ctl, s);
+    if (with_rho) return launch_t<true, __nv_bfloat16>(tm, y, lse, BH, T, causal, sm_count, work_counter, ctl, s);
+    return launch_t<false, __nv_bfloat16>(tm, y, lse, BH, T, causal, sm_count, work_counter, ctl, s);
 }
 
 }  // namespace plx

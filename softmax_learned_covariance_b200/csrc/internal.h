@@ -34,7 +34,15 @@ DecodePlan plan_decode(int B, int H, int Tcap, int d, int sm_count);
 size_t decode_partials_bytes(int B, int H, int d, const DecodePlan &p);
 cudaError_t launch_decode(const void *q, const void *rho, const void *kc, const void *vc, const int *seqlens,
                           void *y, float *lse, int B, int H, int Tcap, int d, int out_dtype, const DecodePlan &p,
-                          float *partials, cudaStream_t s);
+                          float *partials, int sm_count, const DeviceCtl &ctl, cudaStream_t s);
+
+// Wait policy and test hooks from the environment (PARALLAX_WAIT_TIMEOUT_MS,
+// PARALLAX_DEBUG_FLAGS) around the given device error word.  No allocation.
+DeviceCtl ctl_from_env(int *err);
+
+// Device error word of the no-allocation decode entry point on the current
+// device, or nullptr if that entry point has not been set up there.
+int *noalloc_error_word();
 
 // tcgen05 GEMM for rho = x W_R, scattered per head
 cudaError_t launch_rho_proj(const CUtensorMap &tm_x, const CUtensorMap &tm_w, void *rho, int B, int T, int d_model,
@@ -44,7 +52,10 @@ cudaError_t launch_rho_proj(const CUtensorMap &tm_x, const CUtensorMap &tm_w, vo
 struct FwdTensorMaps {
     CUtensorMap q, k, r, v16;
 };
+// work_counter: one device int, reset by the launch (stream-ordered) and used as the
+// persistent grid's atomic item counter.
 cudaError_t launch_fwd_sm100(const FwdTensorMaps &tm, bool with_rho, void *y, float *lse, int B, int H, int T,
-                             int d, int causal, int out_dtype, int sm_count, const DeviceCtl &ctl, cudaStream_t s);
+                             int d, int causal, int out_dtype, int sm_count, int *work_counter, const DeviceCtl &ctl,
+                             cudaStream_t s);
 
 }  // namespace plx

@@ -129,7 +129,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         uint32_t local = 0;
         for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++local) {
             const uint32_t ab = local & 1;
-            if (!mbar_wait(smem_u32(&bars->acc_full[ab]), (local >> 1) & 1, wc)) break;
+            // warp-uniform outcome: tcgen05.ld below is .sync.aligned
+            if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->acc_full[ab]), (local >> 1) & 1, wc))) break;
             tc_fence_after();
             const int m0 = (t / n_tiles) * BM, n0 = (t % n_tiles) * BN;
             const int m = m0 + row_in_tile;
