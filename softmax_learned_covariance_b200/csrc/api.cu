@@ -196,10 +196,11 @@ int parallax_fwd(const void *q, const void *k, const void *v, const void *rho, v
 
     FwdTensorMaps tm;
     const uint64_t dims[3] = {(uint64_t)d, (uint64_t)T, (uint64_t)B * H};
-    const uint32_t box_q[3] = {64, 128, 1}, box_k[3] = {64, 64, 1};
+    // boxes: 64 head-dim columns (128 B, the swizzle span) x {128 query rows, 128 keys, 64 keys}
+    const uint32_t box_q[3] = {64, 128, 1}, box_k[3] = {64, 128, 1}, box_v[3] = {64, 64, 1};
     if ((st = encode(&tm.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, 3, dims, box_q, 2))) return st;
     if ((st = encode(&tm.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k, 3, dims, box_k, 2))) return st;
-    if ((st = encode(&tm.v16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, v16, 3, dims, box_k, 2))) return st;
+    if ((st = encode(&tm.v16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, v16, 3, dims, box_v, 2))) return st;
     if (rho) {
         if ((st = encode(&tm.r, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rho, 3, dims, box_q, 2))) return st;
     } else {

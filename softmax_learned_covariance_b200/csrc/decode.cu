@@ -7,7 +7,7 @@
 // then reads v_j once and accumulates both o and m.  Per token: 8d flops for
 // 4d bytes of K and V.
 //
-// Work is cut into units of (b, h, chunk of tokens).  A grid of 8 small CTAs
+// Work is cut into units of (b, h, chunk of tokens).  A grid of 16 small CTAs
 // per SM strides over the units, so ragged sequence lengths balance without a
 // host-side read of seqlens, and 32 resident warps per SM keep enough 16-byte
 // loads in flight to cover HBM latency.  Within a unit the tokens are taken in
@@ -25,15 +25,17 @@
 namespace plx {
 namespace {
 
-// Measured on B200 (bench shape B=64 H=16 ctx 4096): 4-warp CTAs with 8 of them
-// resident per SM (64 registers per thread) stream at 5.27 TB/s, against 4.5 TB/s
-// for 8-warp CTAs at 3 per SM and 3.6-3.8 TB/s for a TMA-ring variant whose
-// consumer warps were latency bound per block.
-constexpr int NW = 4;            // warps per CTA
+// Measured on B200 (bench shape B=64 H=16 ctx 4096): 2-warp CTAs with 16 of them
+// resident per SM (64 registers per thread) stream at 5.50 TB/s, 4-warp CTAs at
+// 8 per SM at 5.26 TB/s, 8-warp CTAs at 3 per SM at 4.5 TB/s, and a TMA-ring
+// variant whose consumer warps were latency bound per block at 3.6-3.8 TB/s.
+// Small CTAs keep the __syncthreads-separated phases of one CTA from idling the
+// SM: the other CTAs' loads are in flight meanwhile.
+constexpr int NW = 2;            // warps per CTA
 constexpr int NTHREADS = NW * 32;
 constexpr int SUB = 512;         // tokens staged per sub-chunk
 constexpr int UNROLL = 4;        // 16-byte loads in flight per lane per pass step
-constexpr int MIN_BLOCKS = 8;    // resident CTAs per SM the register budget targets
+constexpr int MIN_BLOCKS = 16;   // resident CTAs per SM the register budget targets
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 
@@ -221,36 +223,43 @@ __global__ void __launch_bounds__(NTHREADS, MIN_BLOCKS) k_decode_split(
             sm.red_s[2][warp] = asum;
         }
         __syncthreads();
-        if (tid < D) {
-            float l = 0.f, ab = 0.f, o = 0.f, m = 0.f;
+        {
+            float l = 0.f, ab = 0.f;
 #pragma unroll
             for (int w = 0; w < NW; ++w) {
                 l += sm.red_s[1][w];
                 ab += sm.red_s[2][w];
             }
+            float *P = partials + ((size_t)bh * nsplit + split) * (2 * D + 3);
+            // one output dimension per thread, striding when the CTA is narrower than d
+            for (int e = tid; e < D; e += NTHREADS) {
+                float o = 0.f, m = 0.f;
 #pragma unroll
-            for (int s = 0; s < GROUPS; ++s) {
-                o += sm.red_o[s][tid];
-                m += sm.red_m[s][tid];
-            }
-            if (nsplit == 1) {
-                float out = 0.f;
-                if (l > 0.f) {
-                    const float inv = 1.0f / l;
-                    const float oo = o * inv;
-                    out = oo - (m * inv - oo * (ab * inv));
+                for (int s = 0; s < GROUPS; ++s) {
+                    o += sm.red_o[s][e];
+                    m += sm.red_m[s][e];
                 }
-                store_out<Tout>(y + bh * D + tid, out);
-                if (lse != nullptr && tid == 0) lse[bh] = l > 0.f ? (mu + log2f(l)) * LN2 : -INFINITY;
-            } else {
-                float *P = partials + ((size_t)bh * nsplit + split) * (2 * D + 3);
-                if (tid == 0) {
+                if (nsplit == 1) {
+                    float out = 0.f;
+                    if (l > 0.f) {
+                        const float inv = 1.0f / l;
+                        const float oo = o * inv;
+                        out = oo - (m * inv - oo * (ab * inv));
+                    }
+                    store_out<Tout>(y + bh * D + e, out);
+                } else {
+                    P[3 + e] = o;
+                    P[3 + D + e] = m;
+                }
+            }
+            if (tid == 0) {
+                if (nsplit == 1) {
+                    if (lse != nullptr) lse[bh] = l > 0.f ? (mu + log2f(l)) * LN2 : -INFINITY;
+                } else {
                     P[0] = mu;
                     P[1] = l;
                     P[2] = ab;
                 }
-                P[3 + tid] = o;
-                P[3 + D + tid] = m;
             }
         }
         __syncthreads();
@@ -295,7 +304,7 @@ cudaError_t launch_t(const void *q, const void *rho, const void *kc, const void 
                      cudaStream_t s) {
     const long units = (long)B * H * p.nsplit;
     long grid = units;
-    const long cap = (long)sms * 8;
+    const long cap = (long)sms * MIN_BLOCKS;
     if (grid > cap) grid = cap;
     k_decode_split<D, Tout><<<(unsigned)grid, NTHREADS, 0, s>>>(
         (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)rho, (const __nv_bfloat16 *)kc, (const __nv_bfloat16 *)vc,
@@ -313,8 +322,7 @@ DecodePlan plan_decode(int B, int H, int Tcap, int d, int sm_count) {
     (void)d;
     DecodePlan p;
     const long bh = (long)B * H;
-    const long wave = (long)sm_count * 8;            // resident CTAs of 256 threads
-    const long want_units = 8 * wave;                // several units per CTA for balance
+    const long want_units = 64L * sm_count;          // several units per resident CTA for balance
     long chunk = ((long)Tcap * bh + want_units - 1) / want_units;
     chunk = ((chunk + 255) / 256) * 256;
     if (chunk < 256) chunk = 256;

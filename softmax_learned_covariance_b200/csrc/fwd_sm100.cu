@@ -6,12 +6,13 @@
 // The pages' kernel keeps FlashAttention's KV streaming and reuses each K/V
 // tile for both branches (encorp.ai blog "Integraciones de IA personalizadas
 // tras la atencion Parallax", section "Como cambia Parallax la historia del
-// hardware en GPU Hopper").  Here each 64-key tile is brought into shared
-// memory once by TMA and feeds four UMMAs per 128-row query tile:
+// hardware en GPU Hopper").  Here each 128-key tile is brought into shared
+// memory once by TMA and feeds four UMMA chains per 128-row query tile:
 //   S = Q K^T,  A = R K^T                       (bf16 x bf16 -> fp32, TMEM)
 //   O += P V,   M' += (P o A') V                (fp16 x fp16 -> fp32, TMEM)
-// with P = exp2(S log2e/sqrt(d) - m_ref) and A' = A / 256 staged as fp16 into
-// the TMEM columns of S and A.  fp16 (not bf16) for these operands keeps the
+// with P = exp2(S log2e/sqrt(d) - m_ref) and A' = A / 256, both rounded to
+// fp16 and staged in shared memory (128-byte swizzled, K-major) as the A
+// operands of the P.V UMMAs.  fp16 (not bf16) for these operands keeps the
 // rounding of P o A inside the error budget; the row sums l = sum P and
 // Abar' = sum P o A' are taken from the same rounded fp16 values the MMAs
 // consume, so the result is exact for the rounded weights.  The 1/256 factor
@@ -19,16 +20,25 @@
 // rescales (the running max is only moved when it rises by more than 8 in
 // log2 units; O and M are then rescaled in TMEM).
 //
-// Roles (384 threads, one CTA per SM, persistent over (head, query tile)
+// Why this shape (measured on B200): a tcgen05.mma costs at least ~45-50
+// cycles to issue, so UMMAs with N = 64 run at ~60% of the tensor rate while
+// N >= 128 runs at full rate.  The score UMMAs therefore cover 128 keys.  TMEM
+// then holds S, A, O, M (128 columns each) with no room for a second S/A
+// buffer, so P and P o A' go to shared memory instead: the softmax releases S
+// and A as soon as it has loaded them into registers and the next tile's score
+// UMMAs run while this tile is exponentiated.
+//
+// Roles (576 threads, one CTA per SM, persistent over (head, query tile)
 // items taken longest-first from an atomic work counter):
-//   warp 0      scheduler + TMA producer: Q and R per item, K and V(fp16) rings
-//   warp 1      TMEM owner and single-thread UMMA issuer
-//   warps 4..11 two softmax warpgroups, one query row per thread in each; the
-//               group g handles key columns [32g, 32g+32) of every 64-key tile,
-//               the two exchange their partial row max through shared memory
-// TMEM (512 columns): O [0,128) | M' [128,256) | S0 | A0 | S1 | A1 (64 each),
-// S/A double-buffered so the score UMMAs of tile j+1 run while tile j is
-// exponentiated.
+//   warp 0 lane 0   scheduler + TMA for Q, R (per item) and K (128-key tiles)
+//   warp 0 lane 16  TMA for V (fp16, 64-key stages)
+//   warp 1          TMEM owner and single-thread UMMA issuer
+//   warps 2..17     four softmax warpgroups; group g takes key columns
+//                   [32g, 32g+32) of every tile for all 128 rows, one row per
+//                   thread; the four exchange their partial row max through
+//                   shared memory and an mbarrier
+// Every wait is a bounded mbarrier wait (no named barriers), so a wait that
+// gives up lets every role leave its loop and the kernel return.
 //
 // WITH_RHO = false is the softmax-only instantiation: the same code with the
 // R loads, the A/M UMMAs and the correction arithmetic removed.  With rho = 0
@@ -45,52 +55,66 @@ namespace plx {
 namespace {
 
 constexpr int D = 128;
-constexpr int BM = 128;          // query rows per tile
-constexpr int BN = 64;           // keys per tile
-constexpr int HALF = BN / 2;     // key columns per softmax warpgroup
-constexpr int KST = 4;           // K ring stages
-constexpr int VST = 4;           // V ring stages
-constexpr int SCHED = 4;         // scheduler ring depth (items in flight)
-constexpr int NTHREADS = 384;
-constexpr int NSOFT = 256;       // softmax threads (two warpgroups)
+constexpr int BM = 128;                   // query rows per tile
+constexpr int BN = 128;                   // keys per tile
+constexpr int NGRP = 4;                   // softmax warpgroups
+constexpr int GCOLS = BN / NGRP;          // key columns per group
+constexpr int KST = 2;                    // K ring stages (whole 128-key tiles)
+constexpr int VKEYS = 64;                 // keys per V stage
+constexpr int VST = 2;                    // V ring stages (a stage is reloaded while the next tile's scores run)
+constexpr int VPER = BN / VKEYS;          // V stages per key tile
+constexpr int SCHED = 4;                  // scheduler ring depth (items in flight)
+constexpr int FIRST_SOFT_WARP = 2;
+constexpr int NSOFT_WARPS = NGRP * 4;
+constexpr int NTHREADS = (FIRST_SOFT_WARP + NSOFT_WARPS) * 32;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 constexpr float RESCALE_THRESHOLD = 8.0f;   // log2 units
 constexpr float A_SCALE = 1.0f / 256.0f;
 constexpr float A_UNSCALE = 256.0f;
 
-constexpr int Q_BYTES = BM * D * 2;    // 32 KB, two 64-column halves of [128 x 128 B]
-constexpr int K_BYTES = BN * D * 2;    // 16 KB, two halves of [64 x 128 B]
-constexpr int V_BYTES = BN * D * 2;    // 16 KB fp16, two d-halves of [64 keys x 128 B]
+constexpr int Q_BYTES = BM * D * 2;       // 32 KB: two 64-column halves of [128 rows x 128 B]
+constexpr int K_BYTES = BN * D * 2;       // 32 KB: two halves of [128 keys x 128 B]
+constexpr int V_BYTES = VKEYS * D * 2;    // 16 KB fp16: two d-halves of [64 keys x 128 B]
+constexpr int P_BYTES = BM * BN * 2;      // 32 KB fp16: two key-halves of [128 rows x 128 B]
+
+// shared-memory map (every tile region 1024-byte aligned)
+constexpr int OFF_Q = 0;
+constexpr int OFF_R = OFF_Q + Q_BYTES;
+constexpr int OFF_K = OFF_R + Q_BYTES;
+constexpr int OFF_V = OFF_K + KST * K_BYTES;
+constexpr int OFF_P = OFF_V + VST * V_BYTES;
+constexpr int OFF_PA = OFF_P + P_BYTES;
+constexpr int OFF_BARS = OFF_PA + P_BYTES;
 
 // TMEM column map
-constexpr uint32_t COL_O = 0, COL_M = 128;
-__host__ __device__ constexpr uint32_t col_s(uint32_t b) { return 256 + b * 128; }
-__host__ __device__ constexpr uint32_t col_a(uint32_t b) { return 256 + b * 128 + 64; }
-// fp16 P (or P o A') of key group kk (16 keys) inside the S (or A) buffer: each
-// warpgroup packs its 32 keys into the first 16 columns of its own 32-column half.
-__host__ __device__ constexpr uint32_t col_p16(uint32_t kk) { return (kk >> 1) * 32 + (kk & 1) * 8; }
+constexpr uint32_t COL_S = 0, COL_A = 128, COL_O = 256, COL_M = 384;
 
 constexpr uint32_t IDESC_S = idesc_f16(1, 1, 0, 0, BM, BN);     // bf16 Q/R (K-major) x bf16 K (K-major)
-constexpr uint32_t IDESC_PV = idesc_f16(0, 0, 0, 1, BM, D);     // f16 P (TMEM) x f16 V (MN-major)
+constexpr uint32_t IDESC_PV = idesc_f16(0, 0, 0, 1, BM, D);     // f16 P (K-major) x f16 V (MN-major)
 
 struct __align__(8) Bars {
     uint64_t qr_full, qr_empty;
     uint64_t k_full[KST], k_empty[KST];
     uint64_t v_full[VST], v_empty[VST];
-    uint64_t s_full[2], p_full[2], pv_done[2];
-    uint64_t om_free;
+    uint64_t s_full, a_full;      // score UMMAs of the current tile done
+    uint64_t s_free, a_free;      // softmax has loaded S / A out of TMEM
+    uint64_t p_full;              // P and P o A' are in shared memory
+    uint64_t pv_done;             // P.V UMMAs of the tile done (P buffer reusable)
+    uint64_t om_free;             // epilogue has read O and M
+    uint64_t xchg;                // every softmax warp posted its partial max of the tile
+    uint64_t xread;               // every softmax warp has read the partial maxima of the tile
+    uint64_t esum;                // per item: partial sums posted
     uint64_t sched_full[SCHED], sched_empty[SCHED];
-    uint64_t xchg[2];            // per tile parity: both softmax groups posted their partial max
-    uint64_t esum;               // per item: both softmax groups posted their partial sums
     int sched_item[SCHED];
     uint32_t tmem_base;
     int abort_flag;
-    float red_max[2][2][BM];     // [tile parity][warpgroup][row] partial row max
-    float red_sum[2][2][BM];     // [l or abar'][warpgroup][row] partial sums for the epilogue
+    float red_max[NGRP][BM];      // [group][row] partial row max of the current tile
 };
 
-constexpr size_t SMEM_BYTES = 1024 + 2 * (size_t)Q_BYTES + (size_t)KST * K_BYTES + (size_t)VST * V_BYTES + sizeof(Bars);
+constexpr size_t SMEM_BYTES = (size_t)OFF_BARS + sizeof(Bars);
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+static_assert(2 * NGRP * BM * sizeof(float) <= (size_t)P_BYTES, "epilogue sums alias the P buffer");
 
 struct Item {
     int bh, qt, nkv;
@@ -105,6 +129,12 @@ __device__ __forceinline__ Item item_of(int w, int BH, int nq, int T, int causal
     return it;
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // Bounded wait whose outcome is the same for all 32 lanes (lanes that saw the
 // phase complete still give up if another lane of the warp gave up), so the
 // .sync.aligned tcgen05 instructions that follow are never reached divergently.
@@ -113,13 +143,7 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const W
     return __all_sync(0xffffffffu, got);
 }
 
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-    float r;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-    return r;
-}
-
-// Consumers take the k-th scheduled item from the ring (same sequence in every role).
+// Everyone but the scheduler takes the k-th scheduled item from the ring.
 __device__ __forceinline__ bool next_item(Bars *bars, uint32_t k, int &w, const WaitCtl &wc) {
     const uint32_t s = k % SCHED;
     if (!mbar_wait(smem_u32(&bars->sched_full[s]), (k / SCHED) & 1, wc)) return false;
@@ -127,18 +151,30 @@ __device__ __forceinline__ bool next_item(Bars *bars, uint32_t k, int &w, const 
     return true;
 }
 
+// 16-byte chunk c (0..15 over the 128 keys of a row) of row r in a 128-byte
+// swizzled K-major tile made of two 64-key halves of [128 rows x 128 B].
+__device__ __forceinline__ uint32_t p_chunk_addr(uint32_t base, int r, int c) {
+    return base + (uint32_t)(c >> 3) * (BM * 128) + (uint32_t)r * 128 + (uint32_t)(((c & 7) ^ (r & 7)) << 4);
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
 template <bool WITH_RHO, typename Tout>
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
           const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_v, Tout *__restrict__ y,
           float *__restrict__ lse, int BH, int T, int causal, int *__restrict__ work_counter, DeviceCtl ctl) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sQ = smem;
-    uint8_t *sR = sQ + Q_BYTES;
-    uint8_t *sK = sR + Q_BYTES;
-    uint8_t *sV = sK + KST * K_BYTES;
-    Bars *bars = reinterpret_cast<Bars *>(sV + VST * V_BYTES);
+    extern __shared__ __align__(1024) uint8_t smem[];
+    // The swizzled tiles need a 1024-byte aligned base; there is no slack left
+    // in the budget to realign, so refuse (recorded as a device error) if not.
+    if (smem_u32(smem) & 1023u) {
+        if (threadIdx.x == 0) atomicExch(ctl.err, PARALLAX_ERR_UNSUPPORTED);
+        return;
+    }
+    Bars *bars = reinterpret_cast<Bars *>(smem + OFF_BARS);
+    const uint32_t sbase = smem_u32(smem);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     if (threadIdx.x == 0) {
@@ -152,19 +188,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mbar_init(smem_u32(&bars->v_full[s]), 1);
             mbar_init(smem_u32(&bars->v_empty[s]), 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(smem_u32(&bars->s_full[b]), 1);
-            mbar_init(smem_u32(&bars->p_full[b]), NSOFT);
-            mbar_init(smem_u32(&bars->pv_done[b]), 1);
-        }
-        mbar_init(smem_u32(&bars->om_free), NSOFT);
+        mbar_init(smem_u32(&bars->s_full), 1);
+        mbar_init(smem_u32(&bars->a_full), 1);
+        mbar_init(smem_u32(&bars->s_free), NSOFT_WARPS);
+        mbar_init(smem_u32(&bars->a_free), NSOFT_WARPS);
+        mbar_init(smem_u32(&bars->p_full), NSOFT_WARPS);
+        mbar_init(smem_u32(&bars->pv_done), 1);
+        mbar_init(smem_u32(&bars->om_free), NSOFT_WARPS);
+        mbar_init(smem_u32(&bars->xchg), NSOFT_WARPS);
+        mbar_init(smem_u32(&bars->xread), NSOFT_WARPS);
+        mbar_init(smem_u32(&bars->esum), NSOFT_WARPS);
         for (int s = 0; s < SCHED; ++s) {
             mbar_init(smem_u32(&bars->sched_full[s]), 1);
-            mbar_init(smem_u32(&bars->sched_empty[s]), 1 + NSOFT / 32);   // UMMA thread + one lane per softmax warp
+            mbar_init(smem_u32(&bars->sched_empty[s]), 2 + NSOFT_WARPS);   // UMMA thread, V producer, softmax warps
         }
-        mbar_init(smem_u32(&bars->xchg[0]), NSOFT);
-        mbar_init(smem_u32(&bars->xchg[1]), NSOFT);
-        mbar_init(smem_u32(&bars->esum), NSOFT);
         bars->abort_flag = 0;
         fence_mbar_init();
     }
@@ -182,12 +219,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int items = nq * BH;
 
     if (warp == 0 && lane == 0) {
-        // ============================================= scheduler + producer ==
+        // ===================================== scheduler + Q/R/K producer ==
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
-        tma_prefetch_desc(&tm_v);
         if (WITH_RHO) tma_prefetch_desc(&tm_r);
-        uint32_t kc = 0, vc = 0;
+        uint32_t kc = 0;
         bool ok = true;
         for (uint32_t ic = 0; ok; ++ic) {
             const uint32_t ss = ic % SCHED;
@@ -201,35 +237,45 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (!mbar_wait(smem_u32(&bars->qr_empty), (ic & 1) ^ 1, wc)) break;
             const uint32_t qf = smem_u32(&bars->qr_full);
             mbar_arrive_expect_tx(qf, WITH_RHO ? 2 * Q_BYTES : Q_BYTES);
-            tma_load_3d(smem_u32(sQ), &tm_q, qf, 0, q0, it.bh);
-            tma_load_3d(smem_u32(sQ) + Q_BYTES / 2, &tm_q, qf, 64, q0, it.bh);
+            tma_load_3d(sbase + OFF_Q, &tm_q, qf, 0, q0, it.bh);
+            tma_load_3d(sbase + OFF_Q + Q_BYTES / 2, &tm_q, qf, 64, q0, it.bh);
             if (WITH_RHO) {
-                tma_load_3d(smem_u32(sR), &tm_r, qf, 0, q0, it.bh);
-                tma_load_3d(smem_u32(sR) + Q_BYTES / 2, &tm_r, qf, 64, q0, it.bh);
+                tma_load_3d(sbase + OFF_R, &tm_r, qf, 0, q0, it.bh);
+                tma_load_3d(sbase + OFF_R + Q_BYTES / 2, &tm_r, qf, 64, q0, it.bh);
             }
-            for (int j = 0; j < it.nkv; ++j) {
-                {
-                    const int s = kc % KST;
-                    if (!mbar_wait(smem_u32(&bars->k_empty[s]), ((kc / KST) & 1) ^ 1, wc)) { ok = false; break; }
-                    const uint32_t f = smem_u32(&bars->k_full[s]);
-                    const uint32_t dst = smem_u32(sK + s * K_BYTES);
-                    const bool skip = (ctl.debug_flags & DEBUG_FWD_SKIP_FIRST_K_LOAD) && kc == 0;
-                    if (!skip) {
-                        mbar_arrive_expect_tx(f, K_BYTES);
-                        tma_load_3d(dst, &tm_k, f, 0, j * BN, it.bh);
-                        tma_load_3d(dst + K_BYTES / 2, &tm_k, f, 64, j * BN, it.bh);
-                    }
-                    ++kc;
+            for (int j = 0; j < it.nkv; ++j, ++kc) {
+                const int s = kc % KST;
+                if (!mbar_wait(smem_u32(&bars->k_empty[s]), ((kc / KST) & 1) ^ 1, wc)) { ok = false; break; }
+                const uint32_t f = smem_u32(&bars->k_full[s]);
+                const uint32_t dst = sbase + OFF_K + s * K_BYTES;
+                const bool skip = (ctl.debug_flags & DEBUG_FWD_SKIP_FIRST_K_LOAD) && kc == 0;
+                if (!skip) {
+                    mbar_arrive_expect_tx(f, K_BYTES);
+                    tma_load_3d(dst, &tm_k, f, 0, j * BN, it.bh);
+                    tma_load_3d(dst + K_BYTES / 2, &tm_k, f, 64, j * BN, it.bh);
                 }
-                {
+            }
+        }
+    } else if (warp == 0 && lane == 16) {
+        // ==================================================== V producer ==
+        tma_prefetch_desc(&tm_v);
+        uint32_t vc = 0;
+        bool ok = true;
+        for (uint32_t ic = 0; ok; ++ic) {
+            int w;
+            if (!next_item(bars, ic, w, wc)) break;
+            mbar_arrive(smem_u32(&bars->sched_empty[ic % SCHED]));
+            if (w >= items) break;
+            const Item it = item_of(w, BH, nq, T, causal);
+            for (int j = 0; j < it.nkv && ok; ++j) {
+                for (int vs = 0; vs < VPER; ++vs, ++vc) {
                     const int s = vc % VST;
                     if (!mbar_wait(smem_u32(&bars->v_empty[s]), ((vc / VST) & 1) ^ 1, wc)) { ok = false; break; }
                     const uint32_t f = smem_u32(&bars->v_full[s]);
-                    const uint32_t dst = smem_u32(sV + s * V_BYTES);
+                    const uint32_t dst = sbase + OFF_V + s * V_BYTES;
                     mbar_arrive_expect_tx(f, V_BYTES);
-                    tma_load_3d(dst, &tm_v, f, 0, j * BN, it.bh);
-                    tma_load_3d(dst + V_BYTES / 2, &tm_v, f, 64, j * BN, it.bh);
-                    ++vc;
+                    tma_load_3d(dst, &tm_v, f, 0, j * BN + vs * VKEYS, it.bh);
+                    tma_load_3d(dst + V_BYTES / 2, &tm_v, f, 64, j * BN + vs * VKEYS, it.bh);
                 }
             }
         }
@@ -237,26 +283,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // ==================================================== UMMA issuer ==
         uint32_t kc = 0, vc = 0, G = 0;
         bool ok = true;
-        const uint32_t q_base = smem_u32(sQ), r_base = smem_u32(sR);
+        const uint32_t q_base = sbase + OFF_Q, r_base = sbase + OFF_R;
+        const uint32_t p_base = sbase + OFF_P, pa_base = sbase + OFF_PA;
         auto issue_pv = [&](uint32_t g, bool first, uint32_t icur) -> bool {
-            const uint32_t b = g & 1;
-            if (!mbar_wait(smem_u32(&bars->p_full[b]), (g >> 1) & 1, wc)) return false;
-            const int s = vc % VST;
-            if (!mbar_wait(smem_u32(&bars->v_full[s]), (vc / VST) & 1, wc)) return false;
+            if (!mbar_wait(smem_u32(&bars->p_full), g & 1, wc)) return false;
             if (first && icur > 0)
                 if (!mbar_wait(smem_u32(&bars->om_free), (icur - 1) & 1, wc)) return false;
-            tc_fence_after();
-            const uint32_t vb = smem_u32(sV + s * V_BYTES);
+            for (int vs = 0; vs < VPER; ++vs, ++vc) {
+                const int s = vc % VST;
+                if (!mbar_wait(smem_u32(&bars->v_full[s]), (vc / VST) & 1, wc)) return false;
+                tc_fence_after();
+                const uint32_t vb = sbase + OFF_V + s * V_BYTES;
 #pragma unroll
-            for (int kk = 0; kk < BN / 16; ++kk) {
-                const uint64_t vdesc = sdesc_sw128(vb + kk * 16 * 128, V_BYTES / 2, 1024);
-                const uint32_t acc = (!first || kk > 0) ? 1u : 0u;
-                umma_ts(tmem + COL_O, tmem + col_s(b) + col_p16(kk), vdesc, IDESC_PV, acc);
-                if constexpr (WITH_RHO) umma_ts(tmem + COL_M, tmem + col_a(b) + col_p16(kk), vdesc, IDESC_PV, acc);
+                for (int k2 = 0; k2 < VKEYS / 16; ++k2) {
+                    const int kk = vs * (VKEYS / 16) + k2;     // 16-key step within the tile
+                    const uint32_t poff = (uint32_t)(kk >> 2) * (BM * 128) + (uint32_t)(kk & 3) * 32;
+                    const uint64_t vdesc = sdesc_sw128(vb + k2 * 16 * 128, V_BYTES / 2, 1024);
+                    const uint32_t acc = (first && kk == 0) ? 0u : 1u;
+                    umma_ss(tmem + COL_O, sdesc_sw128(p_base + poff, 16, 1024), vdesc, IDESC_PV, acc);
+                    if constexpr (WITH_RHO)
+                        umma_ss(tmem + COL_M, sdesc_sw128(pa_base + poff, 16, 1024), vdesc, IDESC_PV, acc);
+                }
+                tc_commit(smem_u32(&bars->v_empty[s]));
             }
-            tc_commit(smem_u32(&bars->v_empty[s]));
-            tc_commit(smem_u32(&bars->pv_done[b]));
-            ++vc;
+            tc_commit(smem_u32(&bars->pv_done));
             return true;
         };
         for (uint32_t ic = 0; ok; ++ic) {
@@ -266,39 +316,47 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (w >= items) break;
             const Item it = item_of(w, BH, nq, T, causal);
             if (!mbar_wait(smem_u32(&bars->qr_full), ic & 1, wc)) break;
-            for (int j = 0; j < it.nkv; ++j, ++G) {
-                const uint32_t b = G & 1;
+            for (int j = 0; j < it.nkv; ++j, ++G, ++kc) {
                 const int s = kc % KST;
                 if (!mbar_wait(smem_u32(&bars->k_full[s]), (kc / KST) & 1, wc)) { ok = false; break; }
+                if (G > 0 && !mbar_wait(smem_u32(&bars->s_free), (G - 1) & 1, wc)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t kb = smem_u32(sK + s * K_BYTES);
+                const uint32_t kb = sbase + OFF_K + s * K_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t half = kk >> 2, sub = kk & 3;
-                    const uint64_t qdesc = sdesc_sw128(q_base + half * (Q_BYTES / 2) + sub * 32, 16, 1024);
-                    const uint64_t kdesc = sdesc_sw128(kb + half * (K_BYTES / 2) + sub * 32, 16, 1024);
-                    umma_ss(tmem + col_s(b), qdesc, kdesc, IDESC_S, kk > 0 ? 1u : 0u);
-                    if constexpr (WITH_RHO) {
-                        const uint64_t rdesc = sdesc_sw128(r_base + half * (Q_BYTES / 2) + sub * 32, 16, 1024);
-                        umma_ss(tmem + col_a(b), rdesc, kdesc, IDESC_S, kk > 0 ? 1u : 0u);
+                    const uint32_t off = (uint32_t)(kk >> 2) * (Q_BYTES / 2) + (uint32_t)(kk & 3) * 32;
+                    const uint32_t koff = (uint32_t)(kk >> 2) * (K_BYTES / 2) + (uint32_t)(kk & 3) * 32;
+                    umma_ss(tmem + COL_S, sdesc_sw128(q_base + off, 16, 1024), sdesc_sw128(kb + koff, 16, 1024),
+                            IDESC_S, kk > 0 ? 1u : 0u);
+                }
+                tc_commit(smem_u32(&bars->s_full));
+                if constexpr (WITH_RHO) {
+                    if (G > 0 && !mbar_wait(smem_u32(&bars->a_free), (G - 1) & 1, wc)) { ok = false; break; }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (uint32_t)(kk >> 2) * (Q_BYTES / 2) + (uint32_t)(kk & 3) * 32;
+                        const uint32_t koff = (uint32_t)(kk >> 2) * (K_BYTES / 2) + (uint32_t)(kk & 3) * 32;
+                        umma_ss(tmem + COL_A, sdesc_sw128(r_base + off, 16, 1024), sdesc_sw128(kb + koff, 16, 1024),
+                                IDESC_S, kk > 0 ? 1u : 0u);
                     }
+                    tc_commit(smem_u32(&bars->a_full));
                 }
                 tc_commit(smem_u32(&bars->k_empty[s]));
-                tc_commit(smem_u32(&bars->s_full[b]));
                 if (j == it.nkv - 1) tc_commit(smem_u32(&bars->qr_empty));
-                ++kc;
                 if (j >= 1 && !issue_pv(G - 1, j == 1, ic)) { ok = false; break; }
             }
             if (!ok) break;
             if (!issue_pv(G - 1, it.nkv == 1, ic)) break;
         }
-    } else if (warp >= 4) {
+    } else if (warp >= FIRST_SOFT_WARP) {
         // ============================================ softmax + epilogue ==
-        const int grp = (warp - 4) >> 2;                 // 0: key columns [0,32), 1: [32,64)
-        const int quarter = warp & 3;
+        const int grp = (warp - FIRST_SOFT_WARP) >> 2;   // key columns [32 grp, 32 grp + 32)
+        const int quarter = warp & 3;                    // TMEM lane quarter this warp may access
         const int r = quarter * 32 + lane;               // query row within the tile == TMEM lane
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const float scale_log2 = LOG2E / sqrtf((float)D);
+        const uint32_t p_base = sbase + OFF_P, pa_base = sbase + OFF_PA;
         uint32_t G = 0, ni = 0;   // key tiles and items processed by this CTA
         bool ok = true;
         for (uint32_t ic = 0; ok; ++ic) {
@@ -313,24 +371,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             float m_ref = -INFINITY;
             float l4[4] = {0.f, 0.f, 0.f, 0.f}, a4[4] = {0.f, 0.f, 0.f, 0.f};
             for (int j = 0; j < it.nkv; ++j, ++G) {
-                const uint32_t b = G & 1;
-                if (!warp_wait(smem_u32(&bars->s_full[b]), (G >> 1) & 1, wc)) { ok = false; break; }
+                // ---- scores of this group's 32 keys, then release S ----
+                if (!warp_wait(smem_u32(&bars->s_full), G & 1, wc)) { ok = false; break; }
                 tc_fence_after();
-                uint32_t sr[HALF];
-                uint32_t ar[WITH_RHO ? HALF : 1];
-                tmem_ld16(tmem + lane_off + col_s(b) + grp * HALF, *reinterpret_cast<uint32_t(*)[16]>(&sr[0]));
-                tmem_ld16(tmem + lane_off + col_s(b) + grp * HALF + 16, *reinterpret_cast<uint32_t(*)[16]>(&sr[16]));
-                if constexpr (WITH_RHO) {
-                    tmem_ld16(tmem + lane_off + col_a(b) + grp * HALF, *reinterpret_cast<uint32_t(*)[16]>(&ar[0]));
-                    tmem_ld16(tmem + lane_off + col_a(b) + grp * HALF + 16,
-                              *reinterpret_cast<uint32_t(*)[16]>(&ar[16]));
-                }
+                uint32_t sr[GCOLS];
+                tmem_ld16(tmem + lane_off + COL_S + grp * GCOLS, *reinterpret_cast<uint32_t(*)[16]>(&sr[0]));
+                tmem_ld16(tmem + lane_off + COL_S + grp * GCOLS + 16, *reinterpret_cast<uint32_t(*)[16]>(&sr[16]));
                 tmem_wait_ld();
-                // keys of this tile visible to this row: c < limit
-                const int limit = kvis - (j * BN + grp * HALF);
-                if (limit < HALF) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&bars->s_free));
+                const int limit = kvis - (j * BN + grp * GCOLS);
+                if (limit < GCOLS) {
 #pragma unroll
-                    for (int c = 0; c < HALF; ++c)
+                    for (int c = 0; c < GCOLS; ++c)
                         if (c >= limit) sr[c] = __float_as_uint(-INFINITY);
                 }
                 float mx;
@@ -344,10 +398,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     for (int i = 0; i < 8; ++i) t[i] = fmaxf(t[i], __uint_as_float(sr[i + 24]));
                     mx = fmaxf(fmax3(t[0], t[1], t[2]), fmax3(t[3], t[4], fmax3(t[5], t[6], t[7])));
                 }
-                bars->red_max[G & 1][grp][r] = mx;
-                mbar_arrive(smem_u32(&bars->xchg[G & 1]));
-                if (!warp_wait(smem_u32(&bars->xchg[G & 1]), (G >> 1) & 1, wc)) { ok = false; break; }
-                mx = fmaxf(mx, bars->red_max[G & 1][grp ^ 1][r]) * scale_log2;
+                // ---- row max across the four groups (the previous tile's maxima
+                // must have been read by every group before they are overwritten) ----
+                if (G > 0 && !warp_wait(smem_u32(&bars->xread), (G - 1) & 1, wc)) { ok = false; break; }
+                bars->red_max[grp][r] = mx;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&bars->xchg));
+                if (!warp_wait(smem_u32(&bars->xchg), G & 1, wc)) { ok = false; break; }
+                mx = fmaxf(fmaxf(bars->red_max[0][r], bars->red_max[1][r]),
+                           fmaxf(bars->red_max[2][r], bars->red_max[3][r])) *
+                     scale_log2;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&bars->xread));
                 float alpha = 1.f;
                 bool moved = false;
                 if (mx > m_ref + RESCALE_THRESHOLD) {
@@ -360,15 +422,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     }
                     moved = true;
                 }
-                // O and M' hold earlier tiles of this item: rescale them in TMEM,
-                // each warpgroup its half of the columns.
+                // O and M' hold earlier tiles of this item: once the previous
+                // tile's P.V UMMAs are done, rescale them in TMEM (each group
+                // its 32 columns).
                 if (__any_sync(0xffffffffu, moved && j > 0)) {
-                    const uint32_t gp = G - 1;
-                    if (!warp_wait(smem_u32(&bars->pv_done[gp & 1]), (gp >> 1) & 1, wc)) { ok = false; break; }
+                    if (!warp_wait(smem_u32(&bars->pv_done), (G - 1) & 1, wc)) { ok = false; break; }
                     tc_fence_after();
                     const float f = (moved && j > 0) ? alpha : 1.f;
 #pragma unroll 1
-                    for (int c = grp * 64; c < grp * 64 + 64; c += 16) {
+                    for (int c = grp * GCOLS; c < grp * GCOLS + GCOLS; c += 16) {
                         uint32_t t[16];
                         tmem_ld16(tmem + lane_off + COL_O + c, t);
                         tmem_wait_ld();
@@ -383,52 +445,75 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                             tmem_st16(tmem + lane_off + COL_M + c, t);
                         }
                     }
+                    tmem_wait_st();
                 }
-                // P = exp2(z*log2e - m_ref) as fp16; P o A' as fp16; sums from the rounded values
+                // ---- P = exp2(z log2e - m_ref) as fp16, sums from the rounded values ----
                 const float neg_m = -m_ref;
-                uint32_t pk[HALF / 2];
-                uint32_t pak[WITH_RHO ? HALF / 2 : 1];
+                uint32_t pk[GCOLS / 2];
 #pragma unroll
-                for (int i = 0; i < HALF / 2; ++i) {
+                for (int i = 0; i < GCOLS / 2; ++i) {
                     const float p0 = ex2(fmaf(__uint_as_float(sr[2 * i]), scale_log2, neg_m));
                     const float p1 = ex2(fmaf(__uint_as_float(sr[2 * i + 1]), scale_log2, neg_m));
                     pk[i] = pack_f16x2(p0, p1);
                     l4[i & 3] = add_f16x2_to_f32(l4[i & 3], pk[i]);
-                    if constexpr (WITH_RHO) {
+                }
+                uint32_t pak[WITH_RHO ? GCOLS / 2 : 1];
+                if constexpr (WITH_RHO) {
+                    // ---- correction weights P o A' from this group's 32 a_ij ----
+                    if (!warp_wait(smem_u32(&bars->a_full), G & 1, wc)) { ok = false; break; }
+                    tc_fence_after();
+                    uint32_t ar[GCOLS];
+                    tmem_ld16(tmem + lane_off + COL_A + grp * GCOLS, *reinterpret_cast<uint32_t(*)[16]>(&ar[0]));
+                    tmem_ld16(tmem + lane_off + COL_A + grp * GCOLS + 16,
+                              *reinterpret_cast<uint32_t(*)[16]>(&ar[16]));
+                    tmem_wait_ld();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(&bars->a_free));
+#pragma unroll
+                    for (int i = 0; i < GCOLS / 2; ++i) {
                         const uint32_t ah = pack_f16x2(__uint_as_float(ar[2 * i]) * A_SCALE,
                                                        __uint_as_float(ar[2 * i + 1]) * A_SCALE);
                         pak[i] = hmul2(pk[i], ah);
                         a4[i & 3] = add_f16x2_to_f32(a4[i & 3], pak[i]);
                     }
                 }
-                tmem_st16(tmem + lane_off + col_s(b) + grp * HALF, pk);
-                if constexpr (WITH_RHO) tmem_st16(tmem + lane_off + col_a(b) + grp * HALF, pak);
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(smem_u32(&bars->p_full[b]));
+                // ---- stage P (and P o A') for the P.V UMMAs once the previous ones are done ----
+                if (G > 0 && !warp_wait(smem_u32(&bars->pv_done), (G - 1) & 1, wc)) { ok = false; break; }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int c = grp * 4 + i;
+                    sts128(p_chunk_addr(p_base, r, c), pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                    if constexpr (WITH_RHO)
+                        sts128(p_chunk_addr(pa_base, r, c), pak[4 * i], pak[4 * i + 1], pak[4 * i + 2],
+                               pak[4 * i + 3]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&bars->p_full));
             }
             if (!ok) break;
             // ---------------------------------------------- epilogue --
-            bars->red_sum[0][grp][r] = (l4[0] + l4[1]) + (l4[2] + l4[3]);
-            bars->red_sum[1][grp][r] = (a4[0] + a4[1]) + (a4[2] + a4[3]);
-            mbar_arrive(smem_u32(&bars->esum));
+            // The last P.V UMMAs of this item are done: O and M' are final and the
+            // P buffer is free to hold the partial-sum exchange.
+            if (!warp_wait(smem_u32(&bars->pv_done), (G - 1) & 1, wc)) break;
+            tc_fence_after();
+            float *red_sum = reinterpret_cast<float *>(smem + OFF_P);   // [2][NGRP][BM]
+            red_sum[(0 * NGRP + grp) * BM + r] = (l4[0] + l4[1]) + (l4[2] + l4[3]);
+            red_sum[(1 * NGRP + grp) * BM + r] = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&bars->esum));
             if (!warp_wait(smem_u32(&bars->esum), ni & 1, wc)) break;
             ++ni;
-            const float l = bars->red_sum[0][0][r] + bars->red_sum[0][1][r];
-            const float ab = bars->red_sum[1][0][r] + bars->red_sum[1][1][r];
-            const uint32_t glast = G - 1;
-            if (it.nkv >= 2) {
-                const uint32_t gp = glast - 1;
-                if (!warp_wait(smem_u32(&bars->pv_done[gp & 1]), (gp >> 1) & 1, wc)) break;
-            }
-            if (!warp_wait(smem_u32(&bars->pv_done[glast & 1]), (glast >> 1) & 1, wc)) break;
-            tc_fence_after();
+            const float l = (red_sum[0 * BM + r] + red_sum[1 * BM + r]) + (red_sum[2 * BM + r] + red_sum[3 * BM + r]);
+            const float ab = (red_sum[(NGRP + 0) * BM + r] + red_sum[(NGRP + 1) * BM + r]) +
+                             (red_sum[(NGRP + 2) * BM + r] + red_sum[(NGRP + 3) * BM + r]);
             const float inv_l = 1.0f / l;
             const float abar = ab * inv_l;
             const bool store = qrow < T;
             Tout *yrow = y + ((size_t)it.bh * T + (store ? qrow : 0)) * D;
 #pragma unroll 1
-            for (int c = grp * 64; c < grp * 64 + 64; c += 16) {
+            for (int c = grp * GCOLS; c < grp * GCOLS + GCOLS; c += 16) {
                 uint32_t o[16], mm[16];
                 tmem_ld16(tmem + lane_off + COL_O + c, o);
                 if constexpr (WITH_RHO) tmem_ld16(tmem + lane_off + COL_M + c, mm);
@@ -465,7 +550,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             if (store && grp == 0 && lse != nullptr) lse[(size_t)it.bh * T + qrow] = (m_ref + log2f(l)) * LN2;
             tc_fence_before();
-            mbar_arrive(smem_u32(&bars->om_free));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&bars->om_free));
         }
     }
 

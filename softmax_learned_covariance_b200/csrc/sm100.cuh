@@ -190,6 +190,12 @@ __host__ __device__ constexpr uint32_t idesc_f16(uint32_t a_fmt, uint32_t b_fmt,
            ((M >> 4) << 24);
 }
 
+// Make this thread's generic-proxy shared-memory writes visible to the async
+// proxy (tcgen05.mma operand reads, TMA) before a synchronizing arrive.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ misc --
 __device__ __forceinline__ float ex2(float x) {
     float y;
