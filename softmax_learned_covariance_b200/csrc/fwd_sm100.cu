@@ -11,8 +11,8 @@
 //   S = Q K^T,  A = R K^T                       (bf16 x bf16 -> fp32, TMEM)
 //   O += P V,   M' += (P o A') V                (fp16 x fp16 -> fp32, TMEM)
 // with P = exp2(S log2e/sqrt(d) - m_ref) and A' = A / 256, both rounded to
-// fp16 and staged in shared memory (128-byte swizzled, K-major) as the A
-// operands of the P.V UMMAs.  fp16 (not bf16) for these operands keeps the
+// fp16 and written back into TMEM (over the A columns they were computed from)
+// as the A operands of the P.V UMMAs.  fp16 (not bf16) for these operands keeps the
 // rounding of P o A inside the error budget; the row sums l = sum P and
 // Abar' = sum P o A' are taken from the same rounded fp16 values the MMAs
 // consume, so the result is exact for the rounded weights.  The 1/256 factor
@@ -22,11 +22,13 @@
 //
 // Why this shape (measured on B200): a tcgen05.mma costs at least ~45-50
 // cycles to issue, so UMMAs with N = 64 run at ~60% of the tensor rate while
-// N >= 128 runs at full rate.  The score UMMAs therefore cover 128 keys.  TMEM
-// then holds S, A, O, M (128 columns each) with no room for a second S/A
-// buffer, so P and P o A' go to shared memory instead: the softmax releases S
-// and A as soon as it has loaded them into registers and the next tile's score
-// UMMAs run while this tile is exponentiated.
+// N >= 128 runs at full rate; and shared memory delivers ~128 B/cycle, which
+// an SS UMMA with M = N = 128 already uses up.  The score UMMAs therefore
+// cover 128 keys, and P, P o A' stay in TMEM so the P.V UMMAs read only V from
+// shared memory.  TMEM holds S, A, O, M (128 columns each).  The softmax
+// releases S as soon as it has loaded it, so the next tile's S UMMAs run while
+// this tile is exponentiated; the UMMA order S(j), PV(j-1), A(j) lets A(j)
+// overwrite the columns PV(j-1) has just read.
 //
 // Roles (576 threads, one CTA per SM, persistent over (head, query tile)
 // items taken longest-first from an atomic work counter):
@@ -61,7 +63,7 @@ constexpr int NGRP = 4;                   // softmax warpgroups
 constexpr int GCOLS = BN / NGRP;          // key columns per group
 constexpr int KST = 2;                    // K ring stages (whole 128-key tiles)
 constexpr int VKEYS = 64;                 // keys per V stage
-constexpr int VST = 2;                    // V ring stages (a stage is reloaded while the next tile's scores run)
+constexpr int VST = 4;                    // V ring stages (two tiles ahead)
 constexpr int VPER = BN / VKEYS;          // V stages per key tile
 constexpr int SCHED = 4;                  // scheduler ring depth (items in flight)
 constexpr int FIRST_SOFT_WARP = 2;
@@ -76,45 +78,43 @@ constexpr float A_UNSCALE = 256.0f;
 constexpr int Q_BYTES = BM * D * 2;       // 32 KB: two 64-column halves of [128 rows x 128 B]
 constexpr int K_BYTES = BN * D * 2;       // 32 KB: two halves of [128 keys x 128 B]
 constexpr int V_BYTES = VKEYS * D * 2;    // 16 KB fp16: two d-halves of [64 keys x 128 B]
-constexpr int P_BYTES = BM * BN * 2;      // 32 KB fp16: two key-halves of [128 rows x 128 B]
-
 // shared-memory map (every tile region 1024-byte aligned)
 constexpr int OFF_Q = 0;
 constexpr int OFF_R = OFF_Q + Q_BYTES;
 constexpr int OFF_K = OFF_R + Q_BYTES;
 constexpr int OFF_V = OFF_K + KST * K_BYTES;
-constexpr int OFF_P = OFF_V + VST * V_BYTES;
-constexpr int OFF_PA = OFF_P + P_BYTES;
-constexpr int OFF_BARS = OFF_PA + P_BYTES;
+constexpr int OFF_BARS = OFF_V + VST * V_BYTES;
 
-// TMEM column map
+// TMEM column map.  After group g has loaded its A columns [COL_A + 32g, +32)
+// it writes its fp16 P (16 columns) and P o A' (16 columns) over them.
 constexpr uint32_t COL_S = 0, COL_A = 128, COL_O = 256, COL_M = 384;
+__host__ __device__ constexpr uint32_t col_p(uint32_t kk) { return COL_A + (kk >> 1) * GCOLS + (kk & 1) * 8; }
+constexpr uint32_t PA_SHIFT = GCOLS / 2;   // P o A' sits 16 columns after P
 
 constexpr uint32_t IDESC_S = idesc_f16(1, 1, 0, 0, BM, BN);     // bf16 Q/R (K-major) x bf16 K (K-major)
-constexpr uint32_t IDESC_PV = idesc_f16(0, 0, 0, 1, BM, D);     // f16 P (K-major) x f16 V (MN-major)
+constexpr uint32_t IDESC_PV = idesc_f16(0, 0, 0, 1, BM, D);     // f16 P (TMEM) x f16 V (MN-major)
 
 struct __align__(8) Bars {
     uint64_t qr_full, qr_empty;
     uint64_t k_full[KST], k_empty[KST];
     uint64_t v_full[VST], v_empty[VST];
     uint64_t s_full, a_full;      // score UMMAs of the current tile done
-    uint64_t s_free, a_free;      // softmax has loaded S / A out of TMEM
-    uint64_t p_full;              // P and P o A' are in shared memory
-    uint64_t pv_done;             // P.V UMMAs of the tile done (P buffer reusable)
+    uint64_t s_free;              // softmax has loaded S out of TMEM
+    uint64_t p_full;              // P and P o A' are in TMEM
+    uint64_t pv_done;             // P.V UMMAs of the tile done
     uint64_t om_free;             // epilogue has read O and M
-    uint64_t xchg;                // every softmax warp posted its partial max of the tile
-    uint64_t xread;               // every softmax warp has read the partial maxima of the tile
+    uint64_t xchg[2];             // per tile parity: every softmax warp posted its partial max
     uint64_t esum;                // per item: partial sums posted
     uint64_t sched_full[SCHED], sched_empty[SCHED];
     int sched_item[SCHED];
     uint32_t tmem_base;
     int abort_flag;
-    float red_max[NGRP][BM];      // [group][row] partial row max of the current tile
+    float red_max[2][NGRP][BM];   // [tile parity][group][row] partial row max
+    float red_sum[2][NGRP][BM];   // [l or abar'][group][row] partial sums for the epilogue
 };
 
 constexpr size_t SMEM_BYTES = (size_t)OFF_BARS + sizeof(Bars);
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert(2 * NGRP * BM * sizeof(float) <= (size_t)P_BYTES, "epilogue sums alias the P buffer");
 
 struct Item {
     int bh, qt, nkv;
@@ -151,14 +151,13 @@ __device__ __forceinline__ bool next_item(Bars *bars, uint32_t k, int &w, const 
     return true;
 }
 
-// 16-byte chunk c (0..15 over the 128 keys of a row) of row r in a 128-byte
-// swizzled K-major tile made of two 64-key halves of [128 rows x 128 B].
-__device__ __forceinline__ uint32_t p_chunk_addr(uint32_t base, int r, int c) {
-    return base + (uint32_t)(c >> 3) * (BM * 128) + (uint32_t)r * 128 + (uint32_t)(((c & 7) ^ (r & 7)) << 4);
-}
-
-__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+// d0,d1 = a0,a1 * b + c as one packed fp32x2 FMA.
+__device__ __forceinline__ void ffma2(float &d0, float &d1, float a0, float a1, float b, float c) {
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %4};\n\tmov.b64 rc, {%5, %5};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b), "f"(c));
 }
 
 template <bool WITH_RHO, typename Tout>
@@ -191,12 +190,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_init(smem_u32(&bars->s_full), 1);
         mbar_init(smem_u32(&bars->a_full), 1);
         mbar_init(smem_u32(&bars->s_free), NSOFT_WARPS);
-        mbar_init(smem_u32(&bars->a_free), NSOFT_WARPS);
         mbar_init(smem_u32(&bars->p_full), NSOFT_WARPS);
         mbar_init(smem_u32(&bars->pv_done), 1);
         mbar_init(smem_u32(&bars->om_free), NSOFT_WARPS);
-        mbar_init(smem_u32(&bars->xchg), NSOFT_WARPS);
-        mbar_init(smem_u32(&bars->xread), NSOFT_WARPS);
+        mbar_init(smem_u32(&bars->xchg[0]), NSOFT_WARPS);
+        mbar_init(smem_u32(&bars->xchg[1]), NSOFT_WARPS);
         mbar_init(smem_u32(&bars->esum), NSOFT_WARPS);
         for (int s = 0; s < SCHED; ++s) {
             mbar_init(smem_u32(&bars->sched_full[s]), 1);
@@ -281,10 +279,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
     } else if (warp == 1 && lane == 0) {
         // ==================================================== UMMA issuer ==
+        // Per key tile j of an item: S(j), then PV(j-1), then A(j).  A(j) is
+        // written over the TMEM columns from which PV(j-1) reads P and P o A',
+        // which the in-order tensor pipe makes safe.
         uint32_t kc = 0, vc = 0, G = 0;
         bool ok = true;
         const uint32_t q_base = sbase + OFF_Q, r_base = sbase + OFF_R;
-        const uint32_t p_base = sbase + OFF_P, pa_base = sbase + OFF_PA;
         auto issue_pv = [&](uint32_t g, bool first, uint32_t icur) -> bool {
             if (!mbar_wait(smem_u32(&bars->p_full), g & 1, wc)) return false;
             if (first && icur > 0)
@@ -297,12 +297,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
                 for (int k2 = 0; k2 < VKEYS / 16; ++k2) {
                     const int kk = vs * (VKEYS / 16) + k2;     // 16-key step within the tile
-                    const uint32_t poff = (uint32_t)(kk >> 2) * (BM * 128) + (uint32_t)(kk & 3) * 32;
                     const uint64_t vdesc = sdesc_sw128(vb + k2 * 16 * 128, V_BYTES / 2, 1024);
                     const uint32_t acc = (first && kk == 0) ? 0u : 1u;
-                    umma_ss(tmem + COL_O, sdesc_sw128(p_base + poff, 16, 1024), vdesc, IDESC_PV, acc);
-                    if constexpr (WITH_RHO)
-                        umma_ss(tmem + COL_M, sdesc_sw128(pa_base + poff, 16, 1024), vdesc, IDESC_PV, acc);
+                    umma_ts(tmem + COL_O, tmem + col_p(kk), vdesc, IDESC_PV, acc);
+                    if constexpr (WITH_RHO) umma_ts(tmem + COL_M, tmem + col_p(kk) + PA_SHIFT, vdesc, IDESC_PV, acc);
                 }
                 tc_commit(smem_u32(&bars->v_empty[s]));
             }
@@ -330,9 +328,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                             IDESC_S, kk > 0 ? 1u : 0u);
                 }
                 tc_commit(smem_u32(&bars->s_full));
+                if (j >= 1 && !issue_pv(G - 1, j == 1, ic)) { ok = false; break; }
                 if constexpr (WITH_RHO) {
-                    if (G > 0 && !mbar_wait(smem_u32(&bars->a_free), (G - 1) & 1, wc)) { ok = false; break; }
-                    tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint32_t off = (uint32_t)(kk >> 2) * (Q_BYTES / 2) + (uint32_t)(kk & 3) * 32;
@@ -340,11 +337,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         umma_ss(tmem + COL_A, sdesc_sw128(r_base + off, 16, 1024), sdesc_sw128(kb + koff, 16, 1024),
                                 IDESC_S, kk > 0 ? 1u : 0u);
                     }
-                    tc_commit(smem_u32(&bars->a_full));
                 }
+                tc_commit(smem_u32(&bars->a_full));   // with no correction branch: marks the tile's S + PV issue
                 tc_commit(smem_u32(&bars->k_empty[s]));
                 if (j == it.nkv - 1) tc_commit(smem_u32(&bars->qr_empty));
-                if (j >= 1 && !issue_pv(G - 1, j == 1, ic)) { ok = false; break; }
             }
             if (!ok) break;
             if (!issue_pv(G - 1, it.nkv == 1, ic)) break;
@@ -356,7 +352,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int r = quarter * 32 + lane;               // query row within the tile == TMEM lane
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const float scale_log2 = LOG2E / sqrtf((float)D);
-        const uint32_t p_base = sbase + OFF_P, pa_base = sbase + OFF_PA;
         uint32_t G = 0, ni = 0;   // key tiles and items processed by this CTA
         bool ok = true;
         for (uint32_t ic = 0; ok; ++ic) {
@@ -398,18 +393,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     for (int i = 0; i < 8; ++i) t[i] = fmaxf(t[i], __uint_as_float(sr[i + 24]));
                     mx = fmaxf(fmax3(t[0], t[1], t[2]), fmax3(t[3], t[4], fmax3(t[5], t[6], t[7])));
                 }
-                // ---- row max across the four groups (the previous tile's maxima
-                // must have been read by every group before they are overwritten) ----
-                if (G > 0 && !warp_wait(smem_u32(&bars->xread), (G - 1) & 1, wc)) { ok = false; break; }
-                bars->red_max[grp][r] = mx;
+                // ---- row max across the four groups ----
+                bars->red_max[G & 1][grp][r] = mx;
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&bars->xchg));
-                if (!warp_wait(smem_u32(&bars->xchg), G & 1, wc)) { ok = false; break; }
-                mx = fmaxf(fmaxf(bars->red_max[0][r], bars->red_max[1][r]),
-                           fmaxf(bars->red_max[2][r], bars->red_max[3][r])) *
+                if (lane == 0) mbar_arrive(smem_u32(&bars->xchg[G & 1]));
+                if (!warp_wait(smem_u32(&bars->xchg[G & 1]), (G >> 1) & 1, wc)) { ok = false; break; }
+                mx = fmaxf(fmaxf(bars->red_max[G & 1][0][r], bars->red_max[G & 1][1][r]),
+                           fmaxf(bars->red_max[G & 1][2][r], bars->red_max[G & 1][3][r])) *
                      scale_log2;
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&bars->xread));
                 float alpha = 1.f;
                 bool moved = false;
                 if (mx > m_ref + RESCALE_THRESHOLD) {
@@ -452,62 +443,53 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 uint32_t pk[GCOLS / 2];
 #pragma unroll
                 for (int i = 0; i < GCOLS / 2; ++i) {
-                    const float p0 = ex2(fmaf(__uint_as_float(sr[2 * i]), scale_log2, neg_m));
-                    const float p1 = ex2(fmaf(__uint_as_float(sr[2 * i + 1]), scale_log2, neg_m));
-                    pk[i] = pack_f16x2(p0, p1);
+                    float x0, x1;
+                    ffma2(x0, x1, __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]), scale_log2, neg_m);
+                    pk[i] = pack_f16x2(ex2(x0), ex2(x1));
                     l4[i & 3] = add_f16x2_to_f32(l4[i & 3], pk[i]);
                 }
+                // ---- A columns: their UMMA (and with it the previous tile's P.V
+                // UMMAs, which read the same columns) is done ----
+                if (!warp_wait(smem_u32(&bars->a_full), G & 1, wc)) { ok = false; break; }
+                tc_fence_after();
                 uint32_t pak[WITH_RHO ? GCOLS / 2 : 1];
                 if constexpr (WITH_RHO) {
-                    // ---- correction weights P o A' from this group's 32 a_ij ----
-                    if (!warp_wait(smem_u32(&bars->a_full), G & 1, wc)) { ok = false; break; }
-                    tc_fence_after();
                     uint32_t ar[GCOLS];
                     tmem_ld16(tmem + lane_off + COL_A + grp * GCOLS, *reinterpret_cast<uint32_t(*)[16]>(&ar[0]));
                     tmem_ld16(tmem + lane_off + COL_A + grp * GCOLS + 16,
                               *reinterpret_cast<uint32_t(*)[16]>(&ar[16]));
                     tmem_wait_ld();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(smem_u32(&bars->a_free));
 #pragma unroll
                     for (int i = 0; i < GCOLS / 2; ++i) {
-                        const uint32_t ah = pack_f16x2(__uint_as_float(ar[2 * i]) * A_SCALE,
-                                                       __uint_as_float(ar[2 * i + 1]) * A_SCALE);
-                        pak[i] = hmul2(pk[i], ah);
+                        float a0, a1;
+                        ffma2(a0, a1, __uint_as_float(ar[2 * i]), __uint_as_float(ar[2 * i + 1]), A_SCALE, 0.f);
+                        pak[i] = hmul2(pk[i], pack_f16x2(a0, a1));
                         a4[i & 3] = add_f16x2_to_f32(a4[i & 3], pak[i]);
                     }
                 }
-                // ---- stage P (and P o A') for the P.V UMMAs once the previous ones are done ----
-                if (G > 0 && !warp_wait(smem_u32(&bars->pv_done), (G - 1) & 1, wc)) { ok = false; break; }
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int c = grp * 4 + i;
-                    sts128(p_chunk_addr(p_base, r, c), pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-                    if constexpr (WITH_RHO)
-                        sts128(p_chunk_addr(pa_base, r, c), pak[4 * i], pak[4 * i + 1], pak[4 * i + 2],
-                               pak[4 * i + 3]);
-                }
-                fence_proxy_async_smem();
+                // ---- P and P o A' over this group's A columns, for the P.V UMMAs ----
+                tmem_st16(tmem + lane_off + COL_A + grp * GCOLS, pk);
+                if constexpr (WITH_RHO) tmem_st16(tmem + lane_off + COL_A + grp * GCOLS + PA_SHIFT, pak);
+                tmem_wait_st();
+                tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&bars->p_full));
             }
             if (!ok) break;
             // ---------------------------------------------- epilogue --
-            // The last P.V UMMAs of this item are done: O and M' are final and the
-            // P buffer is free to hold the partial-sum exchange.
-            if (!warp_wait(smem_u32(&bars->pv_done), (G - 1) & 1, wc)) break;
-            tc_fence_after();
-            float *red_sum = reinterpret_cast<float *>(smem + OFF_P);   // [2][NGRP][BM]
-            red_sum[(0 * NGRP + grp) * BM + r] = (l4[0] + l4[1]) + (l4[2] + l4[3]);
-            red_sum[(1 * NGRP + grp) * BM + r] = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+            bars->red_sum[0][grp][r] = (l4[0] + l4[1]) + (l4[2] + l4[3]);
+            bars->red_sum[1][grp][r] = (a4[0] + a4[1]) + (a4[2] + a4[3]);
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&bars->esum));
             if (!warp_wait(smem_u32(&bars->esum), ni & 1, wc)) break;
             ++ni;
-            const float l = (red_sum[0 * BM + r] + red_sum[1 * BM + r]) + (red_sum[2 * BM + r] + red_sum[3 * BM + r]);
-            const float ab = (red_sum[(NGRP + 0) * BM + r] + red_sum[(NGRP + 1) * BM + r]) +
-                             (red_sum[(NGRP + 2) * BM + r] + red_sum[(NGRP + 3) * BM + r]);
+            const float l = (bars->red_sum[0][0][r] + bars->red_sum[0][1][r]) +
+                            (bars->red_sum[0][2][r] + bars->red_sum[0][3][r]);
+            const float ab = (bars->red_sum[1][0][r] + bars->red_sum[1][1][r]) +
+                             (bars->red_sum[1][2][r] + bars->red_sum[1][3][r]);
+            // the last P.V UMMAs of this item are done: O and M' are final
+            if (!warp_wait(smem_u32(&bars->pv_done), (G - 1) & 1, wc)) break;
+            tc_fence_after();
             const float inv_l = 1.0f / l;
             const float abar = ab * inv_l;
             const bool store = qrow < T;
