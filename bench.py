@@ -56,6 +56,13 @@ def decode_bytes(B, H, d, seqlens):
     return kv + B * H * d * 2 * 2 + B * H * d * 4
 
 
+# DRAM bytes per algorithmic byte of the decode kernel, from an ncu capture of
+# the same kernel at B=16 H=16 ctx 8192 (1.0814 GB moved for 1.0740 GB of K/V
+# rows, q, rho and y).  Traffic grows in proportion to the cached tokens read,
+# so a launch's traffic is this ratio times its algorithmic bytes.
+DECODE_TRAFFIC_RATIO = 1.0814 / 1.0740
+
+
 def prefill_pairs(B, H, T, causal=True):
     return B * H * (T * (T + 1) // 2 if causal else T * T)
 
@@ -166,6 +173,64 @@ def run_profile_case(args):
     assert plx.parallax_last_device_error() == 0
     ms = a.elapsed_time(b) / args.steps
     return {"workload": args.workload, "ms": ms, "value": work / (ms * 1e-3) / 1e12, "unit": unit}
+
+
+def run_sweep(args):
+    """Decode sweep: heads 16, d 128, batch x context grid with ragged lengths in
+    [ctx/2, ctx]; cells whose cache exceeds 120 GB are skipped.  Inputs are drawn
+    on the device (seeded); cells small enough to sit in L2 are timed with an
+    L2 flush before every call."""
+    import torch
+
+    import softmax_learned_covariance_b200 as plx
+    from softmax_learned_covariance_b200 import inputs
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    cells = []
+    for idx, b, ctx, nbytes, skipped in inputs.sweep_cells():
+        if skipped:
+            cells.append({"B": b, "ctx": ctx, "skipped": "cache %.0f GB > 120 GB" % (nbytes / 1e9)})
+            continue
+        sl = inputs.ragged_seqlens(b, ctx, 4 + idx)
+        q, r, kc, vc, dsl = inputs.decode_inputs_device(b, 16, ctx, 128, sl, seed=4 + idx, device=dev)
+        y = torch.empty((b, 16, 128), dtype=torch.float32, device=dev)
+        for _ in range(args.warmup):
+            plx.parallax_decode(q, r, kc, vc, dsl, y=y, want_lse=False)
+        torch.cuda.synchronize()
+        # Cells whose cache would stay in the 126 MB L2 are timed call by call
+        # with a 256 MB write between calls; the others stream past L2 anyway.
+        small = nbytes < (256 << 20)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps if small else 1)]
+        if small:
+            for a, e in ev:
+                flush.fill_(1)
+                a.record()
+                plx.parallax_decode(q, r, kc, vc, dsl, y=y, want_lse=False)
+                e.record()
+        else:
+            ev[0][0].record()
+            for _ in range(args.steps):
+                plx.parallax_decode(q, r, kc, vc, dsl, y=y, want_lse=False)
+            ev[0][1].record()
+        torch.cuda.synchronize()
+        assert plx.parallax_last_device_error() == 0
+        ms = sum(a.elapsed_time(e) for a, e in ev) / args.steps
+        nb = decode_bytes(b, 16, 128, sl)
+        gbs = nb / (ms * 1e-3) / 1e9
+        cells.append({"B": b, "ctx": ctx, "ms": round(ms, 4), "GB/s": round(gbs, 1),
+                      "frac": round(gbs / peaks["hbm_gbs"], 4), "bytes": nb, "l2_flushed": small,
+                      "long_context": bool(ctx >= 8192 and b * 16 >= 128)})
+        del q, r, kc, vc, dsl, y
+        torch.cuda.empty_cache()
+    longc = [c["frac"] for c in cells if c.get("long_context")]
+    return {"workload": "decode sweep H=16 d=128, ragged lengths in [ctx/2, ctx]", "unit": "GB/s",
+            "steps": args.steps, "warmup": args.warmup,
+            "peak": peaks["hbm_gbs"], "peak_note": "measured HBM copy bandwidth" if peaks["source"] == "measured"
+            else "fallback", "long_context_min_frac": min(longc) if longc else None, "cells": cells}
 
 
 def run_ours(args, rank, world):
@@ -313,7 +378,8 @@ def run_ours(args, rank, world):
                    "l2": "inputs larger than L2 (2.1 GB decode cache, 0.6 GB prefill tensors); no flush"},
         "roofline": {"bound": "hbm", "kernel": "parallax_decode (split + combine)", "achieved": round(dec_tbs * 1e3 / world, 1),
                      "peak": hbm, "unit": "GB/s", "frac": round(dec_tbs * 1e3 / world / hbm, 4),
-                     "traffic": None, "peak_note": f"{tag} HBM copy bandwidth",
+                     "traffic": round(d_bytes * DECODE_TRAFFIC_RATIO), "traffic_unit": "bytes/launch",
+                     "peak_note": f"{tag} HBM copy bandwidth",
                      "algorithmic_bytes_per_launch": d_bytes, "ms_per_launch": round(dec_ms, 5)},
         "prefill": {"value": round(pre_tfs, 2), "unit": "TFLOP/s", "ms_per_step": round(fwd_ms + rp_ms, 4),
                     "fwd": {"ms": round(fwd_ms, 4), "tflops": round(fwd_tfs / world, 2), "flops": p_flops,
@@ -390,7 +456,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["default", "prefill_long", "profile_fwd", "profile_decode",
+    ap.add_argument("--workload", choices=["default", "prefill_long", "sweep", "profile_fwd", "profile_decode",
                                            "profile_rho"], default="default")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -411,6 +477,9 @@ def main():
 
     if args.workload.startswith("profile_"):
         print(json.dumps(run_profile_case(args)), flush=True)
+        return
+    if args.workload == "sweep":
+        print(json.dumps(run_sweep(args)), flush=True)
         return
     if args.impl == "reference":
         line = run_reference(args, rank, world)
