@@ -11,8 +11,7 @@
 //   S = Q K^T,  A = R K^T                       (bf16 x bf16 -> fp32, TMEM)
 //   O += P V,   M' += (P o A') V                (fp16 x fp16 -> fp32, TMEM)
 // with P = exp2(S log2e/sqrt(d) - m_ref) and A' = A / 256, both rounded to
-// fp16 and written back into TMEM (over the A columns they were computed from)
-// as the A operands of the P.V UMMAs.  fp16 (not bf16) for these operands keeps the
+// fp16 and written back into TMEM as the A operands of the P.V UMMAs.  fp16 (not bf16) for these operands keeps the
 // rounding of P o A inside the error budget; the row sums l = sum P and
 // Abar' = sum P o A' are taken from the same rounded fp16 values the MMAs
 // consume, so the result is exact for the rounded weights.  The 1/256 factor
@@ -25,20 +24,25 @@
 // N >= 128 runs at full rate; and shared memory delivers ~128 B/cycle, which
 // an SS UMMA with M = N = 128 already uses up.  The score UMMAs therefore
 // cover 128 keys, and P, P o A' stay in TMEM so the P.V UMMAs read only V from
-// shared memory.  TMEM holds S, A, O, M (128 columns each).  The softmax
-// releases S as soon as it has loaded it, so the next tile's S UMMAs run while
-// this tile is exponentiated; the UMMA order S(j), PV(j-1), A(j) lets A(j)
-// overwrite the columns PV(j-1) has just read.
+// shared memory.  Issuing is the other limit: the issuing thread shares its SM
+// sub-partition with four softmax warps, and every barrier wait or commit it
+// makes between UMMAs leaves the tensor pipe idle.  Two threads therefore
+// issue: one the score UMMAs S(j), A(j), one the P.V UMMAs, so a wait of one
+// chain never stalls the other.  TMEM holds four 128-column regions: X (S of
+// a tile, then its A), P (the fp16 P and P o A' of a tile), O and M.  The
+// softmax releases X as soon as it has loaded S, and again once it has loaded
+// A; the P region is free once the previous tile's P.V UMMAs are done.
 //
-// Roles (576 threads, one CTA per SM, persistent over (head, query tile)
+// Roles (640 threads, one CTA per SM, persistent over (head, query tile)
 // items taken longest-first from an atomic work counter):
 //   warp 0 lane 0   scheduler + TMA for Q, R (per item) and K (128-key tiles)
-//   warp 0 lane 16  TMA for V (fp16, 64-key stages)
-//   warp 1          TMEM owner and single-thread UMMA issuer
+//   warp 1          TMEM owner; lane 0 issues the score UMMAs S(j), A(j)
 //   warps 2..17     four softmax warpgroups; group g takes key columns
 //                   [32g, 32g+32) of every tile for all 128 rows, one row per
 //                   thread; the four exchange their partial row max through
 //                   shared memory and an mbarrier
+//   warp 18 lane 0  issues the P.V UMMAs
+//   warp 19 lane 0  TMA for V (fp16, 64-key stages)
 // Every wait is a bounded mbarrier wait (no named barriers), so a wait that
 // gives up lets every role leave its loop and the kernel return.
 //
@@ -68,7 +72,9 @@ constexpr int VPER = BN / VKEYS;          // V stages per key tile
 constexpr int SCHED = 4;                  // scheduler ring depth (items in flight)
 constexpr int FIRST_SOFT_WARP = 2;
 constexpr int NSOFT_WARPS = NGRP * 4;
-constexpr int NTHREADS = (FIRST_SOFT_WARP + NSOFT_WARPS) * 32;
+constexpr int PV_WARP = FIRST_SOFT_WARP + NSOFT_WARPS;   // P.V UMMA issuer
+constexpr int V_WARP = PV_WARP + 1;                       // V producer
+constexpr int NTHREADS = (V_WARP + 1) * 32;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 constexpr float RESCALE_THRESHOLD = 8.0f;   // log2 units
@@ -85,10 +91,10 @@ constexpr int OFF_K = OFF_R + Q_BYTES;
 constexpr int OFF_V = OFF_K + KST * K_BYTES;
 constexpr int OFF_BARS = OFF_V + VST * V_BYTES;
 
-// TMEM column map.  After group g has loaded its A columns [COL_A + 32g, +32)
-// it writes its fp16 P (16 columns) and P o A' (16 columns) over them.
-constexpr uint32_t COL_S = 0, COL_A = 128, COL_O = 256, COL_M = 384;
-__host__ __device__ constexpr uint32_t col_p(uint32_t kk) { return COL_A + (kk >> 1) * GCOLS + (kk & 1) * 8; }
+// TMEM column map.  S(j) and then A(j) land in X.  Group g writes its fp16 P
+// (16 columns) and P o A' (16 columns) to [COL_P + 32g, +32).
+constexpr uint32_t COL_X = 0, COL_P = 128, COL_O = 256, COL_M = 384;
+__host__ __device__ constexpr uint32_t col_p(uint32_t kk) { return COL_P + (kk >> 1) * GCOLS + (kk & 1) * 8; }
 constexpr uint32_t PA_SHIFT = GCOLS / 2;   // P o A' sits 16 columns after P
 
 constexpr uint32_t IDESC_S = idesc_f16(1, 1, 0, 0, BM, BN);     // bf16 Q/R (K-major) x bf16 K (K-major)
@@ -98,8 +104,8 @@ struct __align__(8) Bars {
     uint64_t qr_full, qr_empty;
     uint64_t k_full[KST], k_empty[KST];
     uint64_t v_full[VST], v_empty[VST];
-    uint64_t s_full, a_full;      // score UMMAs of the current tile done
-    uint64_t s_free;              // softmax has loaded S out of TMEM
+    uint64_t s_full, a_full;      // S, A UMMAs of the current tile done
+    uint64_t s_free, a_free;      // softmax has loaded S, A out of TMEM
     uint64_t p_full;              // P and P o A' are in TMEM
     uint64_t pv_done;             // P.V UMMAs of the tile done
     uint64_t om_free;             // epilogue has read O and M
@@ -190,6 +196,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_init(smem_u32(&bars->s_full), 1);
         mbar_init(smem_u32(&bars->a_full), 1);
         mbar_init(smem_u32(&bars->s_free), NSOFT_WARPS);
+        mbar_init(smem_u32(&bars->a_free), NSOFT_WARPS);
         mbar_init(smem_u32(&bars->p_full), NSOFT_WARPS);
         mbar_init(smem_u32(&bars->pv_done), 1);
         mbar_init(smem_u32(&bars->om_free), NSOFT_WARPS);
@@ -198,7 +205,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_init(smem_u32(&bars->esum), NSOFT_WARPS);
         for (int s = 0; s < SCHED; ++s) {
             mbar_init(smem_u32(&bars->sched_full[s]), 1);
-            mbar_init(smem_u32(&bars->sched_empty[s]), 2 + NSOFT_WARPS);   // UMMA thread, V producer, softmax warps
+            mbar_init(smem_u32(&bars->sched_empty[s]), 3 + NSOFT_WARPS);   // two UMMA threads, V producer, softmax warps
         }
         bars->abort_flag = 0;
         fence_mbar_init();
@@ -254,7 +261,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
             }
         }
-    } else if (warp == 0 && lane == 16) {
+    } else if (warp == V_WARP && lane == 0) {
         // ==================================================== V producer ==
         tma_prefetch_desc(&tm_v);
         uint32_t vc = 0;
@@ -278,34 +285,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
         }
     } else if (warp == 1 && lane == 0) {
-        // ==================================================== UMMA issuer ==
-        // Per key tile j of an item: S(j), then PV(j-1), then A(j).  A(j) is
-        // written over the TMEM columns from which PV(j-1) reads P and P o A',
-        // which the in-order tensor pipe makes safe.
-        uint32_t kc = 0, vc = 0, G = 0;
+        // ============================================= score UMMA issuer ==
+        // Per key tile j: S(j) into X once the softmax has loaded A(j-1)
+        // (S(j-1) without the correction branch), then A(j) into X once it
+        // has loaded S(j).  The shared-memory descriptors are built once; each
+        // UMMA adds a compile-time offset, keeping this thread's instruction
+        // stream short.
+        uint32_t kc = 0, G = 0;
         bool ok = true;
-        const uint32_t q_base = sbase + OFF_Q, r_base = sbase + OFF_R;
-        auto issue_pv = [&](uint32_t g, bool first, uint32_t icur) -> bool {
-            if (!mbar_wait(smem_u32(&bars->p_full), g & 1, wc)) return false;
-            if (first && icur > 0)
-                if (!mbar_wait(smem_u32(&bars->om_free), (icur - 1) & 1, wc)) return false;
-            for (int vs = 0; vs < VPER; ++vs, ++vc) {
-                const int s = vc % VST;
-                if (!mbar_wait(smem_u32(&bars->v_full[s]), (vc / VST) & 1, wc)) return false;
-                tc_fence_after();
-                const uint32_t vb = sbase + OFF_V + s * V_BYTES;
+        const uint64_t dq = sdesc_sw128(sbase + OFF_Q, 16, 1024);
+        const uint64_t dr = sdesc_sw128(sbase + OFF_R, 16, 1024);
+        const uint64_t dk = sdesc_sw128(sbase + OFF_K, 16, 1024);   // stage s: + s * K_BYTES / 16
+        auto issue_scores = [&](uint64_t da, uint64_t kd) {
 #pragma unroll
-                for (int k2 = 0; k2 < VKEYS / 16; ++k2) {
-                    const int kk = vs * (VKEYS / 16) + k2;     // 16-key step within the tile
-                    const uint64_t vdesc = sdesc_sw128(vb + k2 * 16 * 128, V_BYTES / 2, 1024);
-                    const uint32_t acc = (first && kk == 0) ? 0u : 1u;
-                    umma_ts(tmem + COL_O, tmem + col_p(kk), vdesc, IDESC_PV, acc);
-                    if constexpr (WITH_RHO) umma_ts(tmem + COL_M, tmem + col_p(kk) + PA_SHIFT, vdesc, IDESC_PV, acc);
-                }
-                tc_commit(smem_u32(&bars->v_empty[s]));
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = ((uint32_t)(kk >> 2) * (Q_BYTES / 2) + (uint32_t)(kk & 3) * 32) >> 4;
+                const uint32_t koff = ((uint32_t)(kk >> 2) * (K_BYTES / 2) + (uint32_t)(kk & 3) * 32) >> 4;
+                umma_ss(tmem + COL_X, da + off, kd + koff, IDESC_S, kk > 0 ? 1u : 0u);
             }
-            tc_commit(smem_u32(&bars->pv_done));
-            return true;
         };
         for (uint32_t ic = 0; ok; ++ic) {
             int w;
@@ -317,35 +314,63 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             for (int j = 0; j < it.nkv; ++j, ++G, ++kc) {
                 const int s = kc % KST;
                 if (!mbar_wait(smem_u32(&bars->k_full[s]), (kc / KST) & 1, wc)) { ok = false; break; }
-                if (G > 0 && !mbar_wait(smem_u32(&bars->s_free), (G - 1) & 1, wc)) { ok = false; break; }
+                if (G > 0 && !mbar_wait(smem_u32(WITH_RHO ? &bars->a_free : &bars->s_free), (G - 1) & 1, wc)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
-                const uint32_t kb = sbase + OFF_K + s * K_BYTES;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (uint32_t)(kk >> 2) * (Q_BYTES / 2) + (uint32_t)(kk & 3) * 32;
-                    const uint32_t koff = (uint32_t)(kk >> 2) * (K_BYTES / 2) + (uint32_t)(kk & 3) * 32;
-                    umma_ss(tmem + COL_S, sdesc_sw128(q_base + off, 16, 1024), sdesc_sw128(kb + koff, 16, 1024),
-                            IDESC_S, kk > 0 ? 1u : 0u);
-                }
+                const uint64_t kd = dk + (uint64_t)(s * (K_BYTES >> 4));
+                issue_scores(dq, kd);
                 tc_commit(smem_u32(&bars->s_full));
-                if (j >= 1 && !issue_pv(G - 1, j == 1, ic)) { ok = false; break; }
                 if constexpr (WITH_RHO) {
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (uint32_t)(kk >> 2) * (Q_BYTES / 2) + (uint32_t)(kk & 3) * 32;
-                        const uint32_t koff = (uint32_t)(kk >> 2) * (K_BYTES / 2) + (uint32_t)(kk & 3) * 32;
-                        umma_ss(tmem + COL_A, sdesc_sw128(r_base + off, 16, 1024), sdesc_sw128(kb + koff, 16, 1024),
-                                IDESC_S, kk > 0 ? 1u : 0u);
-                    }
+                    if (!mbar_wait(smem_u32(&bars->s_free), G & 1, wc)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_scores(dr, kd);
+                    tc_commit(smem_u32(&bars->a_full));
                 }
-                tc_commit(smem_u32(&bars->a_full));   // with no correction branch: marks the tile's S + PV issue
                 tc_commit(smem_u32(&bars->k_empty[s]));
                 if (j == it.nkv - 1) tc_commit(smem_u32(&bars->qr_empty));
             }
-            if (!ok) break;
-            if (!issue_pv(G - 1, it.nkv == 1, ic)) break;
         }
-    } else if (warp >= FIRST_SOFT_WARP) {
+    } else if (warp == PV_WARP && lane == 0) {
+        // ============================================== P.V UMMA issuer ==
+        uint32_t vc = 0, G = 0;
+        bool ok = true;
+        const uint64_t dv = sdesc_sw128(sbase + OFF_V, V_BYTES / 2, 1024);   // stage s: + s * V_BYTES / 16
+        for (uint32_t ic = 0; ok; ++ic) {
+            int w;
+            if (!next_item(bars, ic, w, wc)) break;
+            mbar_arrive(smem_u32(&bars->sched_empty[ic % SCHED]));
+            if (w >= items) break;
+            const Item it = item_of(w, BH, nq, T, causal);
+            for (int j = 0; j < it.nkv && ok; ++j, ++G) {
+                if (!mbar_wait(smem_u32(&bars->p_full), G & 1, wc)) { ok = false; break; }
+                // the first tile overwrites O and M': the epilogue of the
+                // previous item must have read them
+                if (j == 0 && ic > 0 && !mbar_wait(smem_u32(&bars->om_free), (ic - 1) & 1, wc)) {
+                    ok = false;
+                    break;
+                }
+                for (int vs = 0; vs < VPER; ++vs, ++vc) {
+                    const int s = vc % VST;
+                    if (!mbar_wait(smem_u32(&bars->v_full[s]), (vc / VST) & 1, wc)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint64_t vd = dv + (uint64_t)(s * (V_BYTES >> 4));
+#pragma unroll
+                    for (int k2 = 0; k2 < VKEYS / 16; ++k2) {
+                        const int kk = vs * (VKEYS / 16) + k2;     // 16-key step within the tile
+                        const uint64_t vdesc = vd + (uint64_t)((k2 * 16 * 128) >> 4);
+                        const uint32_t acc = (j == 0 && kk == 0) ? 0u : 1u;
+                        umma_ts(tmem + COL_O, tmem + col_p(kk), vdesc, IDESC_PV, acc);
+                        if constexpr (WITH_RHO)
+                            umma_ts(tmem + COL_M, tmem + col_p(kk) + PA_SHIFT, vdesc, IDESC_PV, acc);
+                    }
+                    tc_commit(smem_u32(&bars->v_empty[s]));
+                }
+                if (ok) tc_commit(smem_u32(&bars->pv_done));
+            }
+        }
+    } else if (warp >= FIRST_SOFT_WARP && warp < PV_WARP) {
         // ============================================ softmax + epilogue ==
         const int grp = (warp - FIRST_SOFT_WARP) >> 2;   // key columns [32 grp, 32 grp + 32)
         const int quarter = warp & 3;                    // TMEM lane quarter this warp may access
@@ -370,8 +395,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (!warp_wait(smem_u32(&bars->s_full), G & 1, wc)) { ok = false; break; }
                 tc_fence_after();
                 uint32_t sr[GCOLS];
-                tmem_ld16(tmem + lane_off + COL_S + grp * GCOLS, *reinterpret_cast<uint32_t(*)[16]>(&sr[0]));
-                tmem_ld16(tmem + lane_off + COL_S + grp * GCOLS + 16, *reinterpret_cast<uint32_t(*)[16]>(&sr[16]));
+                tmem_ld16(tmem + lane_off + COL_X + grp * GCOLS, *reinterpret_cast<uint32_t(*)[16]>(&sr[0]));
+                tmem_ld16(tmem + lane_off + COL_X + grp * GCOLS + 16, *reinterpret_cast<uint32_t(*)[16]>(&sr[16]));
                 tmem_wait_ld();
                 tc_fence_before();
                 __syncwarp();
@@ -413,12 +438,45 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     }
                     moved = true;
                 }
-                // O and M' hold earlier tiles of this item: once the previous
-                // tile's P.V UMMAs are done, rescale them in TMEM (each group
-                // its 32 columns).
-                if (__any_sync(0xffffffffu, moved && j > 0)) {
+                // ---- P = exp2(z log2e - m_ref) as fp16, sums from the rounded values ----
+                const float neg_m = -m_ref;
+                uint32_t pk[GCOLS / 2];
+#pragma unroll
+                for (int i = 0; i < GCOLS / 2; ++i) {
+                    float x0, x1;
+                    ffma2(x0, x1, __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]), scale_log2, neg_m);
+                    pk[i] = pack_f16x2(ex2(x0), ex2(x1));
+                    l4[i & 3] = add_f16x2_to_f32(l4[i & 3], pk[i]);
+                }
+                uint32_t pak[WITH_RHO ? GCOLS / 2 : 1];
+                if constexpr (WITH_RHO) {
+                    // ---- A of this group's 32 keys, then release X ----
+                    if (!warp_wait(smem_u32(&bars->a_full), G & 1, wc)) { ok = false; break; }
+                    tc_fence_after();
+                    uint32_t ar[GCOLS];
+                    tmem_ld16(tmem + lane_off + COL_X + grp * GCOLS, *reinterpret_cast<uint32_t(*)[16]>(&ar[0]));
+                    tmem_ld16(tmem + lane_off + COL_X + grp * GCOLS + 16,
+                              *reinterpret_cast<uint32_t(*)[16]>(&ar[16]));
+                    tmem_wait_ld();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(&bars->a_free));
+#pragma unroll
+                    for (int i = 0; i < GCOLS / 2; ++i) {
+                        float a0, a1;
+                        ffma2(a0, a1, __uint_as_float(ar[2 * i]), __uint_as_float(ar[2 * i + 1]), A_SCALE, 0.f);
+                        pak[i] = hmul2(pk[i], pack_f16x2(a0, a1));
+                        a4[i & 3] = add_f16x2_to_f32(a4[i & 3], pak[i]);
+                    }
+                }
+                // ---- the previous tile's P.V UMMAs are done: the P region is
+                // free and O, M' hold every earlier tile of this item ----
+                if (G > 0) {
                     if (!warp_wait(smem_u32(&bars->pv_done), (G - 1) & 1, wc)) { ok = false; break; }
                     tc_fence_after();
+                }
+                // a moved reference max rescales O and M' (each group its 32 columns)
+                if (__any_sync(0xffffffffu, moved && j > 0)) {
                     const float f = (moved && j > 0) ? alpha : 1.f;
 #pragma unroll 1
                     for (int c = grp * GCOLS; c < grp * GCOLS + GCOLS; c += 16) {
@@ -436,40 +494,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                             tmem_st16(tmem + lane_off + COL_M + c, t);
                         }
                     }
-                    tmem_wait_st();
                 }
-                // ---- P = exp2(z log2e - m_ref) as fp16, sums from the rounded values ----
-                const float neg_m = -m_ref;
-                uint32_t pk[GCOLS / 2];
-#pragma unroll
-                for (int i = 0; i < GCOLS / 2; ++i) {
-                    float x0, x1;
-                    ffma2(x0, x1, __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]), scale_log2, neg_m);
-                    pk[i] = pack_f16x2(ex2(x0), ex2(x1));
-                    l4[i & 3] = add_f16x2_to_f32(l4[i & 3], pk[i]);
-                }
-                // ---- A columns: their UMMA (and with it the previous tile's P.V
-                // UMMAs, which read the same columns) is done ----
-                if (!warp_wait(smem_u32(&bars->a_full), G & 1, wc)) { ok = false; break; }
-                tc_fence_after();
-                uint32_t pak[WITH_RHO ? GCOLS / 2 : 1];
-                if constexpr (WITH_RHO) {
-                    uint32_t ar[GCOLS];
-                    tmem_ld16(tmem + lane_off + COL_A + grp * GCOLS, *reinterpret_cast<uint32_t(*)[16]>(&ar[0]));
-                    tmem_ld16(tmem + lane_off + COL_A + grp * GCOLS + 16,
-                              *reinterpret_cast<uint32_t(*)[16]>(&ar[16]));
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < GCOLS / 2; ++i) {
-                        float a0, a1;
-                        ffma2(a0, a1, __uint_as_float(ar[2 * i]), __uint_as_float(ar[2 * i + 1]), A_SCALE, 0.f);
-                        pak[i] = hmul2(pk[i], pack_f16x2(a0, a1));
-                        a4[i & 3] = add_f16x2_to_f32(a4[i & 3], pak[i]);
-                    }
-                }
-                // ---- P and P o A' over this group's A columns, for the P.V UMMAs ----
-                tmem_st16(tmem + lane_off + COL_A + grp * GCOLS, pk);
-                if constexpr (WITH_RHO) tmem_st16(tmem + lane_off + COL_A + grp * GCOLS + PA_SHIFT, pak);
+                // ---- P and P o A' into this group's P columns, for the P.V UMMAs ----
+                tmem_st16(tmem + lane_off + COL_P + grp * GCOLS, pk);
+                if constexpr (WITH_RHO) tmem_st16(tmem + lane_off + COL_P + grp * GCOLS + PA_SHIFT, pak);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
