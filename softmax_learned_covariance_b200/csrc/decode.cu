@@ -7,10 +7,12 @@
 // then reads v_j once and accumulates both o and m.  Per token: 8d flops for
 // 4d bytes of K and V.
 //
-// Work is cut into units of (b, h, chunk of tokens).  A grid of 16 small CTAs
-// per SM strides over the units, so ragged sequence lengths balance without a
-// host-side read of seqlens, and 32 resident warps per SM keep enough 16-byte
-// loads in flight to cover HBM latency.  Within a unit the tokens are taken in
+// Work is cut into units of (b, h, chunk of tokens), one small CTA per unit,
+// ordered chunk-major: every head's first chunks (full length for any ragged
+// mix) come first and the short or empty tails last, so the hardware block
+// scheduler balances ragged sequence lengths without a host-side read of
+// seqlens.  16 resident CTAs (32 warps) per SM keep enough 16-byte loads in
+// flight to cover HBM latency.  Within a unit the tokens are taken in
 // sub-chunks of SUB: pass A streams K with 16-byte loads (one token row per
 // D/8 lanes, fully coalesced) and stages z, a in shared memory; the sub-chunk
 // max updates the running max (one rescale per sub-chunk, not per token);
@@ -83,7 +85,7 @@ template <int D, typename Tout>
 __global__ void __launch_bounds__(NTHREADS, MIN_BLOCKS) k_decode_split(
     const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ rho, const __nv_bfloat16 *__restrict__ kc,
     const __nv_bfloat16 *__restrict__ vc, const int *__restrict__ seqlens, Tout *__restrict__ y,
-    float *__restrict__ lse, int H, int Tcap, int chunk, int nsplit, long units, float *__restrict__ partials) {
+    float *__restrict__ lse, int H, int Tcap, int chunk, int nsplit, long BH, float *__restrict__ partials) {
     using S = DecodeSmem<D>;
     constexpr int LPT = S::LPT, TPW = S::TPW, GROUPS = S::GROUPS;
     constexpr int STEP = GROUPS * UNROLL;    // token rows per unrolled step
@@ -95,9 +97,10 @@ __global__ void __launch_bounds__(NTHREADS, MIN_BLOCKS) k_decode_split(
     const int slot = warp * TPW + g;          // token slot within the CTA step
     const float scale_log2 = LOG2E / sqrtf((float)D);
 
+    const long units = BH * nsplit;
     for (long u = blockIdx.x; u < units; u += gridDim.x) {
-        const long bh = u / nsplit;
-        const int split = (int)(u % nsplit);
+        const long bh = u % BH;                 // chunk-major unit order
+        const int split = (int)(u / BH);
         const int b = (int)(bh / H);
         const int L = min(max(seqlens[b], 0), Tcap);   // never read past the cache
         const int t0 = split * chunk;
@@ -302,13 +305,13 @@ template <int D, typename Tout>
 cudaError_t launch_t(const void *q, const void *rho, const void *kc, const void *vc, const int *seqlens, void *y,
                      float *lse, int B, int H, int Tcap, const DecodePlan &p, float *partials, int sms,
                      cudaStream_t s) {
-    const long units = (long)B * H * p.nsplit;
-    long grid = units;
-    const long cap = (long)sms * MIN_BLOCKS;
-    if (grid > cap) grid = cap;
+    (void)sms;
+    const long BH = (long)B * H;
+    const long units = BH * p.nsplit;
+    const long grid = units < 0x7fffffffL ? units : 0x7fffffffL;   // one CTA per unit
     k_decode_split<D, Tout><<<(unsigned)grid, NTHREADS, 0, s>>>(
         (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)rho, (const __nv_bfloat16 *)kc, (const __nv_bfloat16 *)vc,
-        seqlens, (Tout *)y, lse, H, Tcap, p.chunk, p.nsplit, units, partials);
+        seqlens, (Tout *)y, lse, H, Tcap, p.chunk, p.nsplit, BH, partials);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || p.nsplit == 1) return e;
     k_decode_combine<D, Tout><<<(unsigned)(B * H), D, 0, s>>>(partials, seqlens, (Tout *)y, lse, H, p.chunk,
