@@ -269,36 +269,101 @@ __global__ void __launch_bounds__(NTHREADS, MIN_BLOCKS) k_decode_split(
     }
 }
 
-template <int D, typename Tout>
-__global__ void __launch_bounds__(D) k_decode_combine(const float *__restrict__ partials,
-                                                      const int *__restrict__ seqlens, Tout *__restrict__ y,
-                                                      float *__restrict__ lse, int H, int chunk, int nsplit) {
+// Merge of the split partials of one (b, h): mu* = max mu_s, w_s = 2^(mu_s - mu*),
+// then l, abar, O, M are the w-weighted sums and y follows as in the split
+// kernel.  The splits of a head are spread over the warps of the block (two in
+// flight per warp) because a head can have hundreds of them; the warps' sums
+// meet in shared memory.  Few splits take a 4-warp block, many a 16-warp one.
+template <int D, typename Tout, int CMB_WARPS>
+__global__ void __launch_bounds__(CMB_WARPS * 32) k_decode_combine(const float *__restrict__ partials,
+                                                                  const int *__restrict__ seqlens,
+                                                                  Tout *__restrict__ y, float *__restrict__ lse,
+                                                                  int H, int chunk, int nsplit) {
+    constexpr int PER = D / 32;   // head dimensions per lane
+    constexpr int STRIDE = 2 * D + 3;
+    __shared__ float red[CMB_WARPS][2 * D + 2];
+    __shared__ float wmax[CMB_WARPS];
     const long bh = blockIdx.x;
     const int b = (int)(bh / H);
     const int L = min(max(seqlens[b], 0), chunk * nsplit);
     const int nvalid = min(nsplit, (L + chunk - 1) / chunk);
-    const int t = threadIdx.x;
-    const float *P = partials + (size_t)bh * nsplit * (2 * D + 3);
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    const float *P = partials + (size_t)bh * nsplit * STRIDE;
     if (nvalid <= 0) {
-        store_out<Tout>(y + bh * D + t, 0.f);
-        if (lse != nullptr && t == 0) lse[bh] = -INFINITY;
+        for (int e = tid; e < D; e += CMB_WARPS * 32) store_out<Tout>(y + bh * D + e, 0.f);
+        if (lse != nullptr && tid == 0) lse[bh] = -INFINITY;
         return;
     }
+    // ---- mu* ----
     float mu = -INFINITY;
-    for (int s = 0; s < nvalid; ++s) mu = fmaxf(mu, P[(size_t)s * (2 * D + 3)]);
-    float l = 0.f, ab = 0.f, o = 0.f, m = 0.f;
-    for (int s = 0; s < nvalid; ++s) {
-        const float *Ps = P + (size_t)s * (2 * D + 3);
-        const float w = fex2(Ps[0] - mu);
-        l = fmaf(w, Ps[1], l);
-        ab = fmaf(w, Ps[2], ab);
-        o = fmaf(w, Ps[3 + t], o);
-        m = fmaf(w, Ps[3 + D + t], m);
+    for (int s2 = tid; s2 < nvalid; s2 += CMB_WARPS * 32) mu = fmaxf(mu, P[(size_t)s2 * STRIDE]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mu = fmaxf(mu, __shfl_xor_sync(0xffffffffu, mu, off));
+    if (lane == 0) wmax[warp] = mu;
+    __syncthreads();
+    mu = wmax[0];
+#pragma unroll
+    for (int w = 1; w < CMB_WARPS; ++w) mu = fmaxf(mu, wmax[w]);
+    // ---- weighted sums, warp w takes splits w, w + CMB_WARPS, ... ----
+    float l = 0.f, ab = 0.f, o[PER], m[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) o[i] = m[i] = 0.f;
+    int s2 = warp;
+    for (; s2 + CMB_WARPS < nvalid; s2 += 2 * CMB_WARPS) {
+        const float *P0 = P + (size_t)s2 * STRIDE, *P1 = P0 + (size_t)CMB_WARPS * STRIDE;
+        const float h0 = P0[0], h1 = P1[0], l0 = P0[1], l1 = P1[1], a0 = P0[2], a1 = P1[2];
+        float ov0[PER], ov1[PER], mv0[PER], mv1[PER];
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            ov0[i] = P0[3 + lane + 32 * i];
+            ov1[i] = P1[3 + lane + 32 * i];
+            mv0[i] = P0[3 + D + lane + 32 * i];
+            mv1[i] = P1[3 + D + lane + 32 * i];
+        }
+        const float w0 = fex2(h0 - mu), w1 = fex2(h1 - mu);
+        l = fmaf(w1, l1, fmaf(w0, l0, l));
+        ab = fmaf(w1, a1, fmaf(w0, a0, ab));
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            o[i] = fmaf(w1, ov1[i], fmaf(w0, ov0[i], o[i]));
+            m[i] = fmaf(w1, mv1[i], fmaf(w0, mv0[i], m[i]));
+        }
     }
-    const float inv = 1.0f / l;
-    const float oo = o * inv;
-    store_out<Tout>(y + bh * D + t, oo - (m * inv - oo * (ab * inv)));
-    if (lse != nullptr && t == 0) lse[bh] = (mu + log2f(l)) * LN2;
+    if (s2 < nvalid) {
+        const float *P0 = P + (size_t)s2 * STRIDE;
+        const float w0 = fex2(P0[0] - mu);
+        l = fmaf(w0, P0[1], l);
+        ab = fmaf(w0, P0[2], ab);
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            o[i] = fmaf(w0, P0[3 + lane + 32 * i], o[i]);
+            m[i] = fmaf(w0, P0[3 + D + lane + 32 * i], m[i]);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        red[warp][lane + 32 * i] = o[i];
+        red[warp][D + lane + 32 * i] = m[i];
+    }
+    if (lane == 0) {
+        red[warp][2 * D] = l;
+        red[warp][2 * D + 1] = ab;
+    }
+    __syncthreads();
+    if (tid < D) {
+        float lt = 0.f, at = 0.f, ot = 0.f, mt = 0.f;
+#pragma unroll
+        for (int w = 0; w < CMB_WARPS; ++w) {
+            lt += red[w][2 * D];
+            at += red[w][2 * D + 1];
+            ot += red[w][tid];
+            mt += red[w][D + tid];
+        }
+        const float inv = 1.0f / lt;
+        const float oo = ot * inv;
+        store_out<Tout>(y + bh * D + tid, oo - (mt * inv - oo * (at * inv)));
+        if (lse != nullptr && tid == 0) lse[bh] = (mu + log2f(lt)) * LN2;
+    }
 }
 
 template <int D, typename Tout>
@@ -314,8 +379,12 @@ cudaError_t launch_t(const void *q, const void *rho, const void *kc, const void 
         seqlens, (Tout *)y, lse, H, Tcap, p.chunk, p.nsplit, BH, partials);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || p.nsplit == 1) return e;
-    k_decode_combine<D, Tout><<<(unsigned)(B * H), D, 0, s>>>(partials, seqlens, (Tout *)y, lse, H, p.chunk,
-                                                              p.nsplit);
+    if (p.nsplit <= 16)
+        k_decode_combine<D, Tout, 4><<<(unsigned)(B * H), 4 * 32, 0, s>>>(partials, seqlens, (Tout *)y, lse, H,
+                                                                          p.chunk, p.nsplit);
+    else
+        k_decode_combine<D, Tout, 16><<<(unsigned)(B * H), 16 * 32, 0, s>>>(partials, seqlens, (Tout *)y, lse, H,
+                                                                            p.chunk, p.nsplit);
     return cudaGetLastError();
 }
 
@@ -325,10 +394,14 @@ DecodePlan plan_decode(int B, int H, int Tcap, int d, int sm_count) {
     (void)d;
     DecodePlan p;
     const long bh = (long)B * H;
-    const long want_units = 64L * sm_count;          // several units per resident CTA for balance
-    long chunk = ((long)Tcap * bh + want_units - 1) / want_units;
-    chunk = ((chunk + 255) / 256) * 256;
-    if (chunk < 256) chunk = 256;
+    // About 64 units per SM (4 waves of resident CTAs) so the block scheduler
+    // can balance ragged lengths; chunks are multiples of 128 tokens (a unit's
+    // partial state is 2d + 3 floats, ~1% of a 128-token chunk's K/V bytes).
+    const long want_units = 64L * sm_count;
+    long nsplit = want_units / bh;
+    if (nsplit < 1) nsplit = 1;
+    long chunk = ((long)Tcap + nsplit - 1) / nsplit;
+    chunk = ((chunk + 127) / 128) * 128;
     if (chunk >= Tcap) chunk = Tcap;                 // one unit per sequence
     p.chunk = (int)chunk;
     p.nsplit = (int)(((long)Tcap + chunk - 1) / chunk);

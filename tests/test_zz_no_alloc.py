@@ -74,7 +74,10 @@ def test_noalloc_rejects_shapes_beyond_the_static_scratch():
     B, H, Tcap, d = 512, 16, 2048, 128
     need = plx.parallax_decode_workspace_bytes(B, H, Tcap, d)
     if need <= _scratch_limit():
-        pytest.skip("this device's split plan fits the static scratch for the probe shape")
+        # The split plan aims at ~64 units per SM, so the partials stay near
+        # 64 * SMs * (2d + 3) * 4 bytes (9.8 MB on 148 SMs) for every shape and
+        # the rejection is out of reach on such a device.
+        pytest.skip("the split plan keeps every shape's partials within the static scratch on this device")
     kc = torch.empty((B, H, Tcap, d), dtype=torch.bfloat16, device=DEV)
     small = torch.empty((B, H, d), dtype=torch.bfloat16, device=DEV)
     y = torch.empty((B, H, d), dtype=torch.float32, device=DEV)
