@@ -353,6 +353,8 @@ def run_ours(args, rank, world):
         e2e_pre = {"value": world * (p_flops + r_flops) / (e_ms / ksteps * 1e-3) / 1e12, "unit": "TFLOP/s",
                    "h2d_bytes_per_step": h2d_p, "d2h_bytes_per_step": yp.numel() * 4, "steps": ksteps}
 
+    extras = measure_extras(args, stream, barrier, world, peaks, pc, dpq, dpk, dpv, yp, lp, fwd_ms)
+
     dec_tbs = world * d_bytes / (dec_ms * 1e-3) / 1e12
     fwd_tfs = world * p_flops / (fwd_ms * 1e-3) / 1e12
     pre_tfs = world * (p_flops + r_flops) / ((fwd_ms + rp_ms) * 1e-3) / 1e12
@@ -391,11 +393,83 @@ def run_ours(args, rank, world):
                                  "frac": round(rp_tfs / world / bf16, 4)},
                     "e2e": e2e_pre},
         "e2e": e2e,
+        "decode_paged": extras["decode_paged"],
+        "softmax_only_fwd": extras["softmax_only_fwd"],
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
         "peaks": peaks,
     }
     return line
+
+
+PAGED_CFG = dict(B=64, Hq=32, Hkv=8, page_size=64, ctx=4096, d=128)
+
+
+def measure_extras(args, stream, barrier, world, peaks, pc, dpq, dpk, dpv, yp, lp, fwd_ms):
+    """Measurements beside the step (not part of it, not in its timed region):
+    the paged grouped-head decode, and the softmax-only instantiation of the
+    prefill on the same inputs (the compute-matched reference point)."""
+    import torch
+
+    import softmax_learned_covariance_b200 as plx
+
+    dev = dpq.device
+
+    def timed(fn, n):
+        for _ in range(args.warmup):
+            fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        barrier()
+        ms = torch.tensor([a.elapsed_time(b) / n], dtype=torch.float64, device=dev)
+        if world > 1:
+            import torch.distributed as dist
+            dist.all_reduce(ms, op=dist.ReduceOp.MAX)
+        return float(ms.item())
+
+    # ---- paged KV cache, grouped query heads ----
+    c = PAGED_CFG
+    g = torch.Generator(device=dev)
+    g.manual_seed(11)
+    mp = c["ctx"] // c["page_size"]
+    npages = c["B"] * mp
+
+    def randn_bf16(shape, scale=1.0):
+        return (torch.randn(shape, generator=g, device=dev, dtype=torch.float32) * scale).to(torch.bfloat16)
+
+    q = randn_bf16((c["B"], c["Hq"], c["d"]))
+    r = randn_bf16((c["B"], c["Hq"], c["d"]), 0.05)
+    kp = randn_bf16((npages, c["Hkv"], c["page_size"], c["d"]))
+    vp = randn_bf16((npages, c["Hkv"], c["page_size"], c["d"]))
+    table = torch.randperm(npages, generator=g, device=dev).to(torch.int32).view(c["B"], mp)
+    sl = torch.full((c["B"],), c["ctx"], dtype=torch.int32, device=dev)
+    y = torch.empty((c["B"], c["Hq"], c["d"]), dtype=torch.float32, device=dev)
+    with torch.cuda.stream(stream):
+        p_ms = timed(lambda: plx.parallax_decode_paged(q, r, kp, vp, table, sl, y=y, want_lse=False, stream=stream),
+                     args.steps)
+    assert plx.parallax_last_device_error(stream) == 0
+    uniq = c["B"] * c["Hkv"] * c["ctx"] * c["d"] * 2 * 2 + c["B"] * c["Hq"] * c["d"] * (2 + 2 + 4)
+    gbs = uniq / (p_ms * 1e-3) / 1e9
+    paged = {"config": dict(c), "ms": round(p_ms, 4), "unit": "GB/s", "value": round(world * gbs, 1),
+             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                          "frac": round(gbs / peaks["hbm_gbs"], 4), "unit": "GB/s",
+                          "bytes": "unique K/V rows + q, rho, y; the 4 query heads of a KV head re-read its rows "
+                                   "through L2"}}
+    del q, r, kp, vp, table, sl, y
+
+    # ---- softmax-only forward on the prefill inputs ----
+    with torch.cuda.stream(stream):
+        s_ms = timed(lambda: plx.parallax_fwd(dpq, dpk, dpv, None, y=yp, lse=lp, stream=stream), args.steps)
+    pairs = prefill_pairs(pc["B"], pc["H"], pc["T"])
+    s_tf = 4 * pc["d"] * pairs / (s_ms * 1e-3) / 1e12
+    smx = {"ms": round(s_ms, 4), "tflops": round(s_tf, 2), "flops": 4 * pc["d"] * pairs,
+           "parallax_over_softmax_time": round(fwd_ms / s_ms, 3),
+           "note": "rho = NULL instantiation of the same kernel (2 of the 4 GEMMs); same inputs and shape"}
+    return {"decode_paged": paged, "softmax_only_fwd": smx}
 
 
 # --------------------------------------------------------------------------- #

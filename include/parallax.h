@@ -63,7 +63,8 @@ typedef enum {
     PARALLAX_ERR_DTYPE = 4,          /* unsupported dtype or dtype pair */
     PARALLAX_ERR_UNSUPPORTED = 5,    /* valid request this build does not serve */
     PARALLAX_ERR_CUDA = 6,           /* a CUDA runtime/driver call failed */
-    PARALLAX_ERR_DEVICE_TIMEOUT = 7  /* a device-side wait gave up */
+    PARALLAX_ERR_DEVICE_TIMEOUT = 7, /* a device-side wait gave up */
+    PARALLAX_ERR_DEVICE_INDEX = 8    /* a device-side index (a page id) was out of range */
 } parallax_status_t;
 
 /*
@@ -127,6 +128,38 @@ PARALLAX_API int parallax_decode_ex(const void *q, const void *rho, const void *
                        const int *seqlens, void *y, float *lse, int B, int H, int Tcap, int d,
                        int in_dtype, int out_dtype, void *workspace, size_t workspace_bytes,
                        parallax_stream_t stream);
+
+/*
+ * parallax_decode_paged -- parallax_decode over a paged KV cache with grouped
+ * query heads.
+ *
+ * The operator per query head is the one of parallax_decode (zubnet.ai news
+ * item on Parallax, paragraph 2).  The pages describe neither paging nor
+ * grouped heads; these are the layouts serving engines keep their caches in:
+ * the cache is a pool of fixed-size pages that a per-sequence table maps, and
+ * G = Hq / Hkv consecutive query heads share one key/value head (query head h
+ * reads KV head h / G).
+ *
+ *   q, rho         : [B, Hq, d] bf16.
+ *   kpages, vpages : [num_pages, Hkv, page_size, d] bf16.
+ *   block_table    : DEVICE int32 [B, max_pages]; token t of sequence b is row
+ *                    t % page_size of page block_table[b * max_pages + t / page_size].
+ *                    Entries a sequence does not reach are not read.  An entry
+ *                    outside [0, num_pages) that is reached is not followed: its
+ *                    rows read as zero and the device error word is set to
+ *                    PARALLAX_ERR_DEVICE_INDEX (see parallax_last_device_error).
+ *   seqlens        : DEVICE int32 [B], 0 <= seqlens[b] <= max_pages * page_size.
+ *   y              : [B, Hq, d] of out_dtype (F32 or BF16); lse [B, Hq] fp32 or NULL.
+ *   B, Hkv >= 1; Hq a multiple of Hkv; page_size a power of two in [16, 4096];
+ *   max_pages, num_pages >= 1; d in {64, 128}; in_dtype BF16.
+ * Split partials use the library's scratch, sized as
+ * parallax_decode_workspace_bytes(B, Hq, max_pages * page_size, d).  Calls
+ * sharing the library's scratch must be ordered on the device.
+ */
+PARALLAX_API int parallax_decode_paged(const void *q, const void *rho, const void *kpages, const void *vpages,
+                                       const int *block_table, const int *seqlens, void *y, float *lse, int B,
+                                       int Hq, int Hkv, int page_size, int max_pages, int num_pages, int d,
+                                       int in_dtype, int out_dtype, parallax_stream_t stream);
 
 /*
  * parallax_decode_noalloc -- parallax_decode that never allocates device memory.

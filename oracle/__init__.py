@@ -16,6 +16,9 @@ Parity status of each function (how it is pinned, see ``tests/test_oracle_pins.p
                             difference derivative of library SDPA, explicit
                             covariance matrix, invariants)
   rho_proj                : pinned (library matmul, one-hot rows)
+  decode_paged            : pinned to decode, a layout change only (identity page
+                            table on a contiguous cache, permuted pages, grouped
+                            heads equal to replicated key/value heads)
 """
 from __future__ import annotations
 
@@ -126,6 +129,35 @@ class Oracle:
             raise ValueError(f"oracle_decode rejected its arguments (code {rc})")
         return y, lse
 
+    def decode_paged(self, q, rho, kpages, vpages, block_table, seqlens, bh_list=None):
+        """Decode over a paged cache with grouped query heads.
+
+        q, rho: [B, Hq, d]; kpages, vpages: [num_pages, Hkv, page_size, d];
+        block_table: [B, max_pages]; seqlens: [B].  Token t of sequence b is
+        row t % page_size of page block_table[b, t // page_size], and query
+        head h reads key/value head h // (Hq // Hkv).  The layout is undone
+        here -- each head's rows are gathered into the contiguous [B, Hq, Tcap, d]
+        cache of ``decode`` -- and the operator is ``decode``'s.
+        """
+        q, rho = _f64(q), _f64(rho)
+        kp, vp = np.asarray(kpages), np.asarray(vpages)
+        B, Hq, d = q.shape
+        num_pages, Hkv, ps, _ = kp.shape
+        bt = np.asarray(block_table, dtype=np.int64)
+        sl = np.ascontiguousarray(seqlens, dtype=np.int32)
+        max_pages = bt.shape[1]
+        group = Hq // Hkv
+        tcap = max_pages * ps
+        kc = np.zeros((B, Hq, tcap, d), np.float64)
+        vc = np.zeros((B, Hq, tcap, d), np.float64)
+        for b in range(B):
+            t = np.arange(int(sl[b]))
+            pages, rows = bt[b, t // ps], t % ps
+            # [L, Hkv, d] -> [Hkv, L, d] -> query heads h = kv head * group + g
+            kc[b, :, :t.size] = np.repeat(kp[pages, :, rows].transpose(1, 0, 2), group, axis=0)
+            vc[b, :, :t.size] = np.repeat(vp[pages, :, rows].transpose(1, 0, 2), group, axis=0)
+        return self.decode(q, rho, kc, vc, sl, bh_list)
+
     def rho_proj(self, x, W_R, H: int, d: int, bt_list=None):
         """rho [B,H,T,d] = per-head slices of x @ W_R; or rho[n,H,d] for token rows bt_list."""
         x, W_R = _f64(x), _f64(W_R)
@@ -181,6 +213,10 @@ def fwd_rows(q, k, v, rho, rows, causal: bool = True):
 
 def decode(q, rho, kcache, vcache, seqlens, bh_list=None):
     return default().decode(q, rho, kcache, vcache, seqlens, bh_list)
+
+
+def decode_paged(q, rho, kpages, vpages, block_table, seqlens, bh_list=None):
+    return default().decode_paged(q, rho, kpages, vpages, block_table, seqlens, bh_list)
 
 
 def rho_proj(x, W_R, H: int, d: int, bt_list=None):

@@ -21,7 +21,7 @@ import os
 import threading
 
 __all__ = [
-    "ParallaxError", "lib", "parallax_fwd", "parallax_decode", "parallax_decode_ex",
+    "ParallaxError", "lib", "parallax_fwd", "parallax_decode", "parallax_decode_ex", "parallax_decode_paged",
     "parallax_rho_proj", "parallax_decode_workspace_bytes", "parallax_last_device_error",
     "parallax_strerror", "parallax_device_sm_count", "LIB_PATH", "F32", "BF16",
 ]
@@ -51,6 +51,7 @@ def lib() -> ctypes.CDLL:
             L.parallax_fwd.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, P]
             L.parallax_decode.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, P]
             L.parallax_decode_ex.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, P, S, P]
+            L.parallax_decode_paged.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, P]
             L.parallax_decode_workspace_bytes.argtypes = [I, I, I, I]
             L.parallax_decode_workspace_bytes.restype = S
             L.parallax_rho_proj.argtypes = [P, P, P, I, I, I, I, I, I, P]
@@ -58,7 +59,8 @@ def lib() -> ctypes.CDLL:
             L.parallax_strerror.restype = ctypes.c_char_p
             L.parallax_last_device_error.argtypes = [P]
             L.parallax_device_sm_count.argtypes = []
-            for f in (L.parallax_fwd, L.parallax_decode, L.parallax_decode_ex, L.parallax_rho_proj,
+            for f in (L.parallax_fwd, L.parallax_decode, L.parallax_decode_ex, L.parallax_decode_paged,
+                      L.parallax_rho_proj,
                       L.parallax_last_device_error, L.parallax_device_sm_count):
                 f.restype = I
             _lib = L
@@ -171,6 +173,34 @@ def parallax_decode_ex(q, rho, kcache, vcache, seqlens, workspace, out_dtype=Non
                                   _ptr(lse), B, H, Tcap, d, _dtype_code(q.dtype), _dtype_code(y.dtype),
                                   _ptr(workspace), nbytes, _stream(stream))
     _check(st, "parallax_decode_ex")
+    return y, lse
+
+
+def parallax_decode_paged(q, rho, kpages, vpages, block_table, seqlens, out_dtype=None, y=None, lse=None,
+                          stream=None, want_lse: bool = True):
+    """Decode over a paged cache with grouped query heads.
+
+    q, rho: [B, Hq, d]; kpages, vpages: [num_pages, Hkv, page_size, d];
+    block_table: int32 [B, max_pages] and seqlens: int32 [B], both on the device.
+    """
+    torch = _torch()
+    for t, n in ((q, "q"), (rho, "rho"), (kpages, "kpages"), (vpages, "vpages"), (block_table, "block_table"),
+                 (seqlens, "seqlens")):
+        _need(t, n)
+    if seqlens.dtype != torch.int32 or block_table.dtype != torch.int32:
+        raise TypeError("seqlens and block_table must be int32")
+    B, Hq, d = q.shape
+    num_pages, Hkv, page_size, _ = kpages.shape
+    max_pages = block_table.shape[1]
+    out_dtype = out_dtype or torch.float32
+    if y is None:
+        y = torch.empty((B, Hq, d), dtype=out_dtype, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    st = lib().parallax_decode_paged(_ptr(q), _ptr(rho), _ptr(kpages), _ptr(vpages), _ptr(block_table),
+                                     _ptr(seqlens), _ptr(y), _ptr(lse), B, Hq, Hkv, page_size, max_pages,
+                                     num_pages, d, _dtype_code(q.dtype), _dtype_code(y.dtype), _stream(stream))
+    _check(st, "parallax_decode_paged")
     return y, lse
 
 

@@ -141,6 +141,7 @@ const char *parallax_strerror(int status) {
         case PARALLAX_ERR_UNSUPPORTED: return "request not served by this build";
         case PARALLAX_ERR_CUDA: return "a CUDA call failed";
         case PARALLAX_ERR_DEVICE_TIMEOUT: return "a device-side wait gave up (bounded wait expired)";
+        case PARALLAX_ERR_DEVICE_INDEX: return "a device-side index (a page id) was out of range";
         default: return "unknown status";
     }
 }
@@ -251,6 +252,35 @@ int parallax_decode(const void *q, const void *rho, const void *kcache, const vo
                     parallax_stream_t stream) {
     return decode_impl(q, rho, kcache, vcache, seqlens, y, lse, B, H, Tcap, d, in_dtype, out_dtype, nullptr, 0, true,
                        stream);
+}
+
+int parallax_decode_paged(const void *q, const void *rho, const void *kpages, const void *vpages,
+                          const int *block_table, const int *seqlens, void *y, float *lse, int B, int Hq, int Hkv,
+                          int page_size, int max_pages, int num_pages, int d, int in_dtype, int out_dtype,
+                          parallax_stream_t stream) {
+    if (!q || !rho || !kpages || !vpages || !block_table || !seqlens || !y) return PARALLAX_ERR_NULL;
+    if (B < 1 || Hkv < 1 || Hq < Hkv || Hq % Hkv != 0 || max_pages < 1 || num_pages < 1 || (d != 64 && d != 128))
+        return PARALLAX_ERR_SHAPE;
+    if (page_size < 16 || page_size > 4096 || (page_size & (page_size - 1)) != 0) return PARALLAX_ERR_SHAPE;
+    int pshift = 0;
+    while ((1 << pshift) < page_size) ++pshift;
+    if ((long long)max_pages * page_size > (1ll << 30)) return PARALLAX_ERR_SHAPE;
+    if ((long long)num_pages * Hkv * page_size * d > (1ll << 40)) return PARALLAX_ERR_SHAPE;
+    if (!aligned16(q) || !aligned16(rho) || !aligned16(kpages) || !aligned16(vpages) || !aligned4(block_table) ||
+        !aligned4(seqlens) || !aligned16(y) || (lse && !aligned4(lse)))
+        return PARALLAX_ERR_ALIGN;
+    if (in_dtype != PARALLAX_BF16 || (out_dtype != PARALLAX_F32 && out_dtype != PARALLAX_BF16))
+        return PARALLAX_ERR_DTYPE;
+    DevState *s = nullptr;
+    int st = get_state(&s);
+    if (st) return st;
+    const int Tcap = max_pages * page_size;
+    const DecodePlan plan = plan_decode(B, Hq, Tcap, d, s->sms);
+    void *ws = nullptr;
+    if ((st = get_workspace(s, decode_partials_bytes(B, Hq, d, plan), &ws))) return st;
+    const PagedKV pg{block_table, max_pages, num_pages, pshift, Hkv, Hq / Hkv};
+    return status_of(launch_decode_paged(q, rho, kpages, vpages, pg, seqlens, y, lse, B, Hq, d, out_dtype, plan,
+                                         static_cast<float *>(ws), make_ctl(s), static_cast<cudaStream_t>(stream)));
 }
 
 int parallax_decode_ex(const void *q, const void *rho, const void *kcache, const void *vcache, const int *seqlens,

@@ -36,6 +36,17 @@ cudaError_t launch_decode(const void *q, const void *rho, const void *kc, const 
                           void *y, float *lse, int B, int H, int Tcap, int d, int out_dtype, const DecodePlan &p,
                           float *partials, int sm_count, const DeviceCtl &ctl, cudaStream_t s);
 
+// Paged KV layout for the decode: pages [num_pages, Hkv, 1 << pshift, d];
+// query head h reads KV head h / group.
+struct PagedKV {
+    const int *table;   // [B, max_pages] page ids (device)
+    int max_pages, num_pages, pshift, Hkv, group;
+};
+cudaError_t launch_decode_paged(const void *q, const void *rho, const void *kpages, const void *vpages,
+                                const PagedKV &pg, const int *seqlens, void *y, float *lse, int B, int Hq, int d,
+                                int out_dtype, const DecodePlan &p, float *partials, const DeviceCtl &ctl,
+                                cudaStream_t s);
+
 // Wait policy and test hooks from the environment (PARALLAX_WAIT_TIMEOUT_MS,
 // PARALLAX_DEBUG_FLAGS) around the given device error word.  No allocation.
 DeviceCtl ctl_from_env(int *err);

@@ -134,6 +134,25 @@ def decode_inputs(B, H, Tcap, d, seqlens=None, rho_scale=0.05, seed=2):
     return q, rho, kc, vc, np.ascontiguousarray(seqlens, dtype=np.int32)
 
 
+def paged_decode_inputs(B, Hq, Hkv, page_size, max_pages, d, seqlens, rho_scale=0.05, seed=6, spare_pages=3):
+    """Paged, grouped-head decode inputs.
+
+    q, rho [B, Hq, d]; kpages, vpages [num_pages, Hkv, page_size, d] with
+    num_pages = B * max_pages + spare_pages; block_table int32 [B, max_pages]
+    holding a random permutation of the page ids (so a sequence's pages are
+    scattered through the pool and some pages belong to no sequence);
+    seqlens int32 [B].
+    """
+    rng = np.random.default_rng(seed)
+    num_pages = B * max_pages + spare_pages
+    q = _bf(rng, (B, Hq, d))
+    rho = _bf(rng, (B, Hq, d), rho_scale)
+    kp = _bf(rng, (num_pages, Hkv, page_size, d))
+    vp = _bf(rng, (num_pages, Hkv, page_size, d))
+    table = rng.permutation(num_pages)[:B * max_pages].reshape(B, max_pages).astype(np.int32)
+    return q, rho, kp, vp, np.ascontiguousarray(table), np.ascontiguousarray(seqlens, dtype=np.int32)
+
+
 def ragged_seqlens(B, ctx, seed):
     """Integer lengths uniform in [ctx/2, ctx] (the decode sweep's ragged mix)."""
     rng = np.random.default_rng(seed + 7919)

@@ -38,7 +38,7 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_strerror_covers_all_codes(L):
-    for code in range(8):
+    for code in range(9):
         s = plx.parallax_strerror(code)
         assert s and s != "unknown status"
     assert plx.parallax_strerror(99) == "unknown status"
@@ -77,6 +77,25 @@ def test_decode_host_validation(L):
     assert dec(kc=MIS) == 3
     assert dec(i=0) == 4
     assert dec(o=7) == 4
+
+
+def test_decode_paged_host_validation(L):
+    def dec(q=A16, rho=A16, kp=A16, vp=A16, bt=A16, sl=A16, y=A16, B=2, Hq=4, Hkv=2, ps=64, mp=4, npg=8, d=128,
+            i=1, o=0):
+        return L.parallax_decode_paged(q, rho, kp, vp, bt, sl, y, None, B, Hq, Hkv, ps, mp, npg, d, i, o, None)
+    assert dec(bt=None) == 1
+    assert dec(vp=None) == 1
+    assert dec(Hq=3) == 2          # not a multiple of Hkv
+    assert dec(Hq=1) == 2          # fewer query heads than KV heads
+    assert dec(ps=48) == 2         # not a power of two
+    assert dec(ps=8) == 2          # below the minimum page size
+    assert dec(ps=8192) == 2
+    assert dec(mp=0) == 2
+    assert dec(npg=0) == 2
+    assert dec(d=96) == 2
+    assert dec(kp=MIS) == 3
+    assert dec(i=0) == 4
+    assert dec(o=5) == 4
 
 
 def test_rho_proj_host_validation(L):

@@ -229,10 +229,58 @@ def pin_rho_projection(orc):
     assert np.array_equal(rs[0], rho[1, :, 1, :]) and np.array_equal(rs[1], rho[0, :, 0, :])
 
 
+def _paged_case(seed, B=3, Hq=4, Hkv=2, ps=4, max_pages=3, d=5):
+    rng = np.random.default_rng(seed)
+    num_pages = B * max_pages + 2
+    q = rng.standard_normal((B, Hq, d))
+    rho = 0.3 * rng.standard_normal((B, Hq, d))
+    kp = rng.standard_normal((num_pages, Hkv, ps, d))
+    vp = rng.standard_normal((num_pages, Hkv, ps, d))
+    table = rng.permutation(num_pages)[:B * max_pages].reshape(B, max_pages)
+    seqlens = np.array([max_pages * ps, 1, ps + 1][:B], np.int32)
+    return q, rho, kp, vp, table, seqlens
+
+
+def pin_paged_layout(orc):
+    """The paged, grouped-head decode is decode on the cache the pages describe:
+    row t of sequence b is row t % page_size of page table[b, t // page_size], and
+    query head h reads key/value head h // (Hq / Hkv).  The contiguous cache is
+    built here row by row, independently of the oracle's gather."""
+    q, rho, kp, vp, table, seqlens = _paged_case(41)
+    B, Hq, d = q.shape
+    _, Hkv, ps, _ = kp.shape
+    group = Hq // Hkv
+    tcap = table.shape[1] * ps
+    kc = np.zeros((B, Hq, tcap, d))
+    vc = np.zeros((B, Hq, tcap, d))
+    for b in range(B):
+        for h in range(Hq):
+            for t in range(int(seqlens[b])):
+                kc[b, h, t] = kp[table[b, t // ps], h // group, t % ps]
+                vc[b, h, t] = vp[table[b, t // ps], h // group, t % ps]
+    y, lse = orc.decode_paged(q, rho, kp, vp, table, seqlens)
+    yr, lr = orc.decode(q, rho, kc, vc, seqlens)
+    assert np.array_equal(y, yr) and np.array_equal(lse, lr)
+    # renaming the physical pages (and the table with them) changes nothing
+    perm = np.random.default_rng(42).permutation(kp.shape[0])
+    inv = np.argsort(perm)
+    y2, _ = orc.decode_paged(q, rho, kp[perm], vp[perm], inv[table], seqlens)
+    assert np.array_equal(y2, y)
+    # grouped heads = the same pool with every key/value head repeated group times
+    y3, _ = orc.decode_paged(q, rho, np.repeat(kp, group, axis=1), np.repeat(vp, group, axis=1), table, seqlens)
+    assert np.array_equal(y3, y)
+    # a page the table does not reach is never read
+    kp4 = kp.copy()
+    unused = sorted(set(range(kp.shape[0])) - set(table.reshape(-1).tolist()))
+    kp4[unused] = np.nan
+    y4, _ = orc.decode_paged(q, rho, kp4, vp, table, seqlens)
+    assert np.array_equal(y4, y)
+
+
 PINS = [pin_softmax_special_case, pin_single_key, pin_two_key_closed_form,
         pin_golden_worked_example, pin_derivative_of_softmax_attention, pin_explicit_covariance,
         pin_one_pass_and_third_form, pin_invariants, pin_rows_and_decode_agree_with_fwd,
-        pin_rho_projection]
+        pin_rho_projection, pin_paged_layout]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -296,3 +344,36 @@ def test_planted_mistakes_are_caught():
     finally:
         shutil.rmtree(tmpdir, ignore_errors=True)
     assert not survivors, f"planted mistakes no pin detects: {survivors}"
+
+
+# The paged decode's gather is Python (oracle/__init__.py); plant mistakes in a
+# copy of that method and require pin_paged_layout to catch each.
+GATHER_MUTANTS = {
+    "page_and_row_swapped": ("pages, rows = bt[b, t // ps], t % ps", "pages, rows = bt[b, t % ps], t // ps"),
+    "heads_interleaved": ("np.repeat(kp[pages, :, rows].transpose(1, 0, 2), group, axis=0)",
+                          "np.tile(kp[pages, :, rows].transpose(1, 0, 2), (group, 1, 1))"),
+    "table_row_of_wrong_sequence": ("pages, rows = bt[b, t // ps], t % ps", "pages, rows = bt[0, t // ps], t % ps"),
+    "v_rows_from_k": ("vc[b, :, :t.size] = np.repeat(vp[pages", "vc[b, :, :t.size] = np.repeat(kp[pages"),
+}
+
+
+def test_planted_gather_mistakes_are_caught():
+    import inspect
+    import textwrap
+
+    src = textwrap.dedent(inspect.getsource(oracle.Oracle.decode_paged))
+    survivors = []
+    for name, (old, new) in GATHER_MUTANTS.items():
+        assert src.count(old) == 1, f"mutation {name}: pattern not found"
+        ns = {"np": np, "_f64": oracle._f64}
+        exec(compile(src.replace(old, new), f"<{name}>", "exec"), ns)
+        orc = oracle.default()
+        mutant = type("MutantOracle", (oracle.Oracle,), {"decode_paged": ns["decode_paged"]})
+        m = mutant.__new__(mutant)
+        m.__dict__.update(orc.__dict__)
+        try:
+            pin_paged_layout(m)
+            survivors.append(name)
+        except (AssertionError, ValueError, IndexError):
+            pass
+    assert not survivors, f"planted gather mistakes pin_paged_layout misses: {survivors}"
