@@ -275,7 +275,7 @@ int parallax_decode_paged(const void *q, const void *rho, const void *kpages, co
     int st = get_state(&s);
     if (st) return st;
     const int Tcap = max_pages * page_size;
-    const DecodePlan plan = plan_decode(B, Hq, Tcap, d, s->sms);
+    const DecodePlan plan = plan_decode_paged(B, Hq, Hkv, Tcap, d, s->sms);
     void *ws = nullptr;
     if ((st = get_workspace(s, decode_partials_bytes(B, Hq, d, plan), &ws))) return st;
     const PagedKV pg{block_table, max_pages, num_pages, pshift, Hkv, Hq / Hkv};

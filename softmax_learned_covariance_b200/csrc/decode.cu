@@ -406,6 +406,18 @@ __global__ void __launch_bounds__(CMB_WARPS * 32) k_decode_combine(const float *
     }
 }
 
+template <int D, typename Tout>
+cudaError_t launch_combine(const float *partials, const int *seqlens, void *y, float *lse, int B, int H,
+                           const DecodePlan &p, cudaStream_t s) {
+    if (p.nsplit <= 16)
+        k_decode_combine<D, Tout, 4><<<(unsigned)(B * H), 4 * 32, 0, s>>>(partials, seqlens, (Tout *)y, lse, H,
+                                                                          p.chunk, p.nsplit);
+    else
+        k_decode_combine<D, Tout, 16><<<(unsigned)(B * H), 16 * 32, 0, s>>>(partials, seqlens, (Tout *)y, lse, H,
+                                                                            p.chunk, p.nsplit);
+    return cudaGetLastError();
+}
+
 template <int D, typename Tout, bool PAGED>
 cudaError_t launch_t(const void *q, const void *rho, const void *kc, const void *vc, const int *seqlens, void *y,
                      float *lse, int B, int H, int Tcap, const DecodePlan &p, float *partials, const PagedKV &pg,
@@ -418,13 +430,7 @@ cudaError_t launch_t(const void *q, const void *rho, const void *kc, const void 
         seqlens, (Tout *)y, lse, H, Tcap, p.chunk, p.nsplit, BH, partials, pg, err);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || p.nsplit == 1) return e;
-    if (p.nsplit <= 16)
-        k_decode_combine<D, Tout, 4><<<(unsigned)(B * H), 4 * 32, 0, s>>>(partials, seqlens, (Tout *)y, lse, H,
-                                                                          p.chunk, p.nsplit);
-    else
-        k_decode_combine<D, Tout, 16><<<(unsigned)(B * H), 16 * 32, 0, s>>>(partials, seqlens, (Tout *)y, lse, H,
-                                                                            p.chunk, p.nsplit);
-    return cudaGetLastError();
+    return launch_combine<D, Tout>(partials, seqlens, y, lse, B, H, p, s);
 }
 
 template <bool PAGED>
@@ -476,13 +482,29 @@ cudaError_t launch_decode(const void *q, const void *rho, const void *kc, const 
                              s);
 }
 
+DecodePlan plan_decode_paged(int B, int Hq, int Hkv, int Tcap, int d, int sm_count) {
+    const int group = Hq / Hkv;
+    // grouped heads: one tensor-core unit serves up to 8 query heads of a KV head
+    if (group >= 2) return plan_decode(B, Hkv * ((group + 7) / 8), Tcap, d, sm_count);
+    return plan_decode(B, Hq, Tcap, d, sm_count);
+}
+
 cudaError_t launch_decode_paged(const void *q, const void *rho, const void *kpages, const void *vpages,
                                 const PagedKV &pg, const int *seqlens, void *y, float *lse, int B, int Hq, int d,
                                 int out_dtype, const DecodePlan &p, float *partials, const DeviceCtl &ctl,
                                 cudaStream_t s) {
     const int Tcap = pg.max_pages << pg.pshift;
-    return launch_any<true>(q, rho, kpages, vpages, seqlens, y, lse, B, Hq, Tcap, d, out_dtype, p, partials, pg,
-                            ctl.err, s);
+    if (pg.group < 2)
+        return launch_any<true>(q, rho, kpages, vpages, seqlens, y, lse, B, Hq, Tcap, d, out_dtype, p, partials, pg,
+                                ctl.err, s);
+    cudaError_t e = launch_decode_gqa_split(q, rho, kpages, vpages, pg, seqlens, y, lse, B, Hq, d, out_dtype, p,
+                                            partials, ctl.err, s);
+    if (e != cudaSuccess || p.nsplit == 1) return e;
+    if (d == 64)
+        return out_dtype == PARALLAX_F32 ? launch_combine<64, float>(partials, seqlens, y, lse, B, Hq, p, s)
+                                         : launch_combine<64, __nv_bfloat16>(partials, seqlens, y, lse, B, Hq, p, s);
+    return out_dtype == PARALLAX_F32 ? launch_combine<128, float>(partials, seqlens, y, lse, B, Hq, p, s)
+                                     : launch_combine<128, __nv_bfloat16>(partials, seqlens, y, lse, B, Hq, p, s);
 }
 
 }  // namespace plx

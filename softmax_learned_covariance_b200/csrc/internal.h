@@ -42,6 +42,13 @@ struct PagedKV {
     const int *table;   // [B, max_pages] page ids (device)
     int max_pages, num_pages, pshift, Hkv, group;
 };
+// Split plan of the paged decode for the kernel that serves this head grouping.
+DecodePlan plan_decode_paged(int B, int Hq, int Hkv, int Tcap, int d, int sm_count);
+// Tensor-core split kernel for grouped heads (Hq / Hkv >= 2); writes the same
+// partials (or y when nsplit == 1) as the split decode kernel.
+cudaError_t launch_decode_gqa_split(const void *q, const void *rho, const void *kpages, const void *vpages,
+                                    const PagedKV &pg, const int *seqlens, void *y, float *lse, int B, int Hq, int d,
+                                    int out_dtype, const DecodePlan &p, float *partials, int *err, cudaStream_t s);
 cudaError_t launch_decode_paged(const void *q, const void *rho, const void *kpages, const void *vpages,
                                 const PagedKV &pg, const int *seqlens, void *y, float *lse, int B, int Hq, int d,
                                 int out_dtype, const DecodePlan &p, float *partials, const DeviceCtl &ctl,

@@ -96,3 +96,16 @@ def test_paged_gqa_b8_hq16_hkv4_ctx2048_all_heads():
     parity.assert_lse(lse.cpu().numpy(), lr)
     y16, _ = _run(_dev(q, rho, kp, vp, table, sl), out_dtype=torch.bfloat16)
     assert torch.equal(y16, y.to(torch.bfloat16))
+
+
+@pytest.mark.parametrize("group", [3, 8, 12])
+def test_paged_group_sizes_beyond_one_tile(group):
+    """Groups that fill a tensor-core tile exactly (8), partly (3) or span two tiles (12)."""
+    B, Hkv, ps, max_pages, d = 3, 2, 32, 24, 128
+    Hq = Hkv * group
+    sl = np.array([ps * max_pages, 5, 400], np.int32)
+    q, rho, kp, vp, table, sl = inputs.paged_decode_inputs(B, Hq, Hkv, ps, max_pages, d, sl, seed=300 + group)
+    y, lse = _run(_dev(q, rho, kp, vp, table, sl))
+    yr, lr = oracle.decode_paged(q.f64, rho.f64, kp.f64, vp.f64, table, sl)
+    parity.assert_bf16_parity(y.cpu().numpy(), yr, 2, f"group {group}")
+    parity.assert_lse(lse.cpu().numpy(), lr)
