@@ -484,8 +484,10 @@ cudaError_t launch_decode(const void *q, const void *rho, const void *kc, const 
 
 DecodePlan plan_decode_paged(int B, int Hq, int Hkv, int Tcap, int d, int sm_count) {
     const int group = Hq / Hkv;
-    // grouped heads: one tensor-core unit serves up to 8 query heads of a KV head
-    if (group >= 2) return plan_decode(B, Hkv * ((group + 7) / 8), Tcap, d, sm_count);
+    // grouped heads: a 4-warp tensor-core unit serves up to 8 query heads of a
+    // KV head; it is sized like four split-kernel units so that each warp
+    // streams enough tiles to amortise its pipeline fill and the final merge
+    if (group >= 2) return plan_decode(B, Hkv * ((group + 7) / 8) * 4, Tcap, d, sm_count);
     return plan_decode(B, Hq, Tcap, d, sm_count);
 }
 

@@ -17,7 +17,7 @@
 //
 // A CTA of 4 warps takes one (sequence, KV head, up to 8 query heads, chunk)
 // unit; each warp streams its own 16-token tiles of the chunk through a
-// 2-stage cp.async ring in shared memory (128-byte-row swizzle, read back with
+// 3-stage cp.async ring in shared memory (128-byte-row swizzle, read back with
 // ldmatrix) and keeps its own online-softmax state; the four states are
 // merged at the end and written as the same partials (or y) as the split
 // kernel, so the split combine applies unchanged.
@@ -32,7 +32,7 @@ namespace {
 
 constexpr int WARPS = 4;
 constexpr int TILE = 16;      // tokens per warp step
-constexpr int STAGES = 2;
+constexpr int STAGES = 3;    // tiles in flight per warp: STAGES - 1
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 
@@ -51,7 +51,9 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+template <int N> __device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 __device__ __forceinline__ void cp_async_wait_0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
@@ -188,13 +190,18 @@ __global__ void __launch_bounds__(WARPS * 32) k_decode_gqa(
             }
         };
 
-        int s = 0;
-        if (warp < ntiles) issue(warp, 0);
-        cp_async_commit();
-        for (int i = warp; i < ntiles; i += WARPS, s ^= 1) {
-            if (i + WARPS < ntiles) issue(i + WARPS, s ^ 1);
+        // this warp's tiles are i = warp + WARPS k; tile k lives in stage k % STAGES
+#pragma unroll
+        for (int k = 0; k < STAGES - 1; ++k) {
+            if (warp + WARPS * k < ntiles) issue(warp + WARPS * k, k);
             cp_async_commit();
-            cp_async_wait_1();
+        }
+        int s = 0;
+        for (int i = warp, k = 0; i < ntiles; i += WARPS, ++k, s = (s + 1 == STAGES) ? 0 : s + 1) {
+            const int inext = i + WARPS * (STAGES - 1);
+            if (inext < ntiles) issue(inext, (s + STAGES - 1) % STAGES);   // the stage computed last iteration
+            cp_async_commit();
+            cp_async_wait<STAGES - 1>();
             __syncwarp();
             const uint8_t *kt = ring + s * GqaSmem<D>::STAGE_BYTES;
             const uint8_t *vt = kt + TILE * D * 2;
@@ -265,7 +272,7 @@ __global__ void __launch_bounds__(WARPS * 32) k_decode_gqa(
                 mma_f16(oacc[j], afr, bf16x2_to_f16x2(v0), bf16x2_to_f16x2(v1));
                 mma_f16(oacc[j + 1], afr, bf16x2_to_f16x2(v2), bf16x2_to_f16x2(v3));
             }
-            __syncwarp();   // the stage is refilled two tiles later
+            __syncwarp();   // this stage is refilled by the next iteration's copies
         }
         cp_async_wait_0();
 
