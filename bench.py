@@ -137,6 +137,7 @@ def run_profile_case(args):
     profile_fwd    : parallax_fwd, B=2 H=16 T=8192 d=128 causal (plus its rho input)
     profile_decode : parallax_decode, B=16 H=16 d=128, 8192-token cache
     profile_rho    : parallax_rho_proj, x [2, 8192, 2048] @ W_R [2048, 2048]
+    profile_paged  : parallax_decode_paged, B=64 Hq=32 Hkv=8, 64-token pages, ctx 4096 (1.07 GB)
     """
     import torch
 
@@ -157,6 +158,24 @@ def run_profile_case(args):
         y = torch.empty((16, 16, 128), dtype=torch.float32, device=dev)
         call = lambda: plx.parallax_decode(q, r, kc, vc, dsl, y=y, want_lse=False)
         work, unit = decode_bytes(16, 16, 128, sl), "TB/s"
+    elif args.workload == "profile_paged":
+        c = PAGED_CFG
+        mp = c["ctx"] // c["page_size"]
+        g = torch.Generator(device=dev)
+        g.manual_seed(11)
+
+        def randn_bf16(shape, scale=1.0):
+            return (torch.randn(shape, generator=g, device=dev, dtype=torch.float32) * scale).to(torch.bfloat16)
+
+        q, r = randn_bf16((c["B"], c["Hq"], c["d"])), randn_bf16((c["B"], c["Hq"], c["d"]), 0.05)
+        kp = randn_bf16((c["B"] * mp, c["Hkv"], c["page_size"], c["d"]))
+        vp = randn_bf16((c["B"] * mp, c["Hkv"], c["page_size"], c["d"]))
+        tb = torch.randperm(c["B"] * mp, generator=g, device=dev).to(torch.int32).view(c["B"], mp)
+        dsl = torch.full((c["B"],), c["ctx"], dtype=torch.int32, device=dev)
+        y = torch.empty((c["B"], c["Hq"], c["d"]), dtype=torch.float32, device=dev)
+        call = lambda: plx.parallax_decode_paged(q, r, kp, vp, tb, dsl, y=y, want_lse=False)
+        work = c["B"] * c["Hkv"] * c["ctx"] * c["d"] * 4 + c["B"] * c["Hq"] * c["d"] * 8
+        unit = "TB/s"
     else:
         x, w = (t.torch().to(dev) for t in inputs.rho_proj_inputs(2, 8192, 2048, 16, 128, seed=3))
         r = torch.empty((2, 16, 8192, 128), dtype=torch.bfloat16, device=dev)
@@ -532,7 +551,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["default", "prefill_long", "sweep", "profile_fwd", "profile_decode",
-                                           "profile_rho"], default="default")
+                                           "profile_rho", "profile_paged"], default="default")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

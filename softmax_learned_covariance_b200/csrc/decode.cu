@@ -168,8 +168,12 @@ __global__ void __launch_bounds__(NTHREADS, MIN_BLOCKS) k_decode_split(
 #pragma unroll
                 for (int x = 0; x < UNROLL; ++x) {
                     const int tok = base + x * GROUPS + slot;
-                    const uint4 *pk = tok < n ? row(kbase, s0 + tok) : nullptr;
-                    kr[x] = pk ? ldg_stream(pk) : make_uint4(0, 0, 0, 0);
+                    if constexpr (PAGED) {
+                        const uint4 *pk = tok < n ? row(kbase, s0 + tok) : nullptr;
+                        kr[x] = pk ? ldg_stream(pk) : make_uint4(0, 0, 0, 0);
+                    } else {
+                        kr[x] = tok < n ? ldg_stream(kbase + (size_t)(s0 + tok) * LPT) : make_uint4(0, 0, 0, 0);
+                    }
                 }
 #pragma unroll
                 for (int x = 0; x < UNROLL; ++x) {
@@ -229,8 +233,12 @@ __global__ void __launch_bounds__(NTHREADS, MIN_BLOCKS) k_decode_split(
 #pragma unroll
                 for (int x = 0; x < UNROLL; ++x) {
                     const int tok = base + x * GROUPS + slot;
-                    const uint4 *pv = tok < n ? row(vbase, s0 + tok) : nullptr;
-                    vr[x] = pv ? ldg_stream(pv) : make_uint4(0, 0, 0, 0);
+                    if constexpr (PAGED) {
+                        const uint4 *pv = tok < n ? row(vbase, s0 + tok) : nullptr;
+                        vr[x] = pv ? ldg_stream(pv) : make_uint4(0, 0, 0, 0);
+                    } else {
+                        vr[x] = tok < n ? ldg_stream(vbase + (size_t)(s0 + tok) * LPT) : make_uint4(0, 0, 0, 0);
+                    }
                 }
 #pragma unroll
                 for (int x = 0; x < UNROLL; ++x) {
