@@ -39,6 +39,28 @@ PREFILL_CFG = dict(B=8, T=4096, H=16, d=128, d_model=2048)
 LONG_CFG = dict(B=1, T=32768, H=16, d=128, d_model=2048)
 
 
+def rank_env():
+    """(rank, world, local_rank) as the launcher (torchrun) sets them; one process per GPU."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(values, world, device):
+    """Element-wise max of per-rank timings over the process group: the slowest rank times the job."""
+    import torch
+
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_rate(units_per_rank, max_ms, world):
+    """Units all ranks processed per second (every rank runs the same work: weak scaling, replicas)."""
+    return world * units_per_rank / (max_ms * 1e-3)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -329,12 +351,7 @@ def run_ours(args, rank, world):
     rp_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
     fwd_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
 
-    # max over ranks
-    vals = torch.tensor([total_ms, dec_ms, rp_ms, fwd_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        import torch.distributed as dist
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    total_ms, dec_ms, rp_ms, fwd_ms = vals.tolist()
+    total_ms, dec_ms, rp_ms, fwd_ms = max_over_ranks([total_ms, dec_ms, rp_ms, fwd_ms], world, dev)
 
     # ---------------- end to end through the public API, host buffers ----------------
     e2e = e2e_pre = None
@@ -353,8 +370,8 @@ def run_ours(args, rank, world):
             yhost.copy_(yd, non_blocking=True)
         t1.record(stream)
         barrier()
-        e_ms = t0.elapsed_time(t1)
-        e2e = {"value": world * d_bytes / (e_ms / ksteps * 1e-3) / 1e12, "unit": "TB/s",
+        e_ms = max_over_ranks([t0.elapsed_time(t1)], world, dev)[0]
+        e2e = {"value": whole_job_rate(d_bytes, e_ms / ksteps, world) / 1e12, "unit": "TB/s",
                "h2d_bytes_per_step": h2d_d, "d2h_bytes_per_step": d2h_d, "steps": ksteps}
         h2d_p = sum(t.numel() * t.element_size() for t in host_pre)
         yph = torch.empty(yp.shape, dtype=torch.float32).pin_memory()
@@ -368,16 +385,16 @@ def run_ours(args, rank, world):
             yph.copy_(yp, non_blocking=True)
         t1.record(stream)
         barrier()
-        e_ms = t0.elapsed_time(t1)
-        e2e_pre = {"value": world * (p_flops + r_flops) / (e_ms / ksteps * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e_ms = max_over_ranks([t0.elapsed_time(t1)], world, dev)[0]
+        e2e_pre = {"value": whole_job_rate(p_flops + r_flops, e_ms / ksteps, world) / 1e12, "unit": "TFLOP/s",
                    "h2d_bytes_per_step": h2d_p, "d2h_bytes_per_step": yp.numel() * 4, "steps": ksteps}
 
     extras = measure_extras(args, stream, barrier, world, peaks, pc, dpq, dpk, dpv, yp, lp, fwd_ms)
 
-    dec_tbs = world * d_bytes / (dec_ms * 1e-3) / 1e12
-    fwd_tfs = world * p_flops / (fwd_ms * 1e-3) / 1e12
-    pre_tfs = world * (p_flops + r_flops) / ((fwd_ms + rp_ms) * 1e-3) / 1e12
-    rp_tfs = world * r_flops / (rp_ms * 1e-3) / 1e12
+    dec_tbs = whole_job_rate(d_bytes, dec_ms, world) / 1e12
+    fwd_tfs = whole_job_rate(p_flops, fwd_ms, world) / 1e12
+    pre_tfs = whole_job_rate(p_flops + r_flops, fwd_ms + rp_ms, world) / 1e12
+    rp_tfs = whole_job_rate(r_flops, rp_ms, world) / 1e12
     hbm = peaks["hbm_gbs"]
     bf16 = peaks["bf16_tflops"]
     tag = "of measured" if peaks["source"] == "measured" else "of fallback"
@@ -444,11 +461,7 @@ def measure_extras(args, stream, barrier, world, peaks, pc, dpq, dpk, dpv, yp, l
             fn()
         b.record(stream)
         barrier()
-        ms = torch.tensor([a.elapsed_time(b) / n], dtype=torch.float64, device=dev)
-        if world > 1:
-            import torch.distributed as dist
-            dist.all_reduce(ms, op=dist.ReduceOp.MAX)
-        return float(ms.item())
+        return max_over_ranks([a.elapsed_time(b) / n], world, dev)[0]
 
     # ---- paged KV cache, grouped query heads ----
     c = PAGED_CFG
@@ -558,15 +571,14 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
+    rank, world, local_rank = rank_env()
     if world > 1 and args.impl == "ours":
         import datetime
 
         import torch
         import torch.distributed as dist
 
-        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
 
     if args.workload.startswith("profile_"):
