@@ -157,6 +157,7 @@ def run_profile_case(args):
     """Small single-kernel loops for ncu captures (inputs still larger than L2, a few GB at most).
 
     profile_fwd    : parallax_fwd, B=2 H=16 T=8192 d=128 causal (plus its rho input)
+    profile_fwd_long : parallax_fwd, B=1 H=16 T=32768 d=128 causal (the long prefill)
     profile_decode : parallax_decode, B=16 H=16 d=128, 8192-token cache
     profile_rho    : parallax_rho_proj, x [2, 8192, 2048] @ W_R [2048, 2048]
     profile_paged  : parallax_decode_paged, B=64 Hq=32 Hkv=8, 64-token pages, ctx 4096 (1.07 GB)
@@ -168,11 +169,12 @@ def run_profile_case(args):
 
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    if args.workload == "profile_fwd":
-        q, k, v, r = (t.torch().to(dev) for t in inputs.fwd_bf16_inputs(2, 16, 8192, 128, seed=3))
+    if args.workload in ("profile_fwd", "profile_fwd_long"):
+        B, T = (2, 8192) if args.workload == "profile_fwd" else (1, 32768)
+        q, k, v, r = (t.torch().to(dev) for t in inputs.fwd_bf16_inputs(B, 16, T, 128, seed=3 if B == 2 else 5))
         y = torch.empty(q.shape, dtype=torch.float32, device=dev)
         call = lambda: plx.parallax_fwd(q, k, v, r, y=y, want_lse=False)
-        work, unit = prefill_flops(2, 16, 8192, 128), "TFLOP/s"
+        work, unit = prefill_flops(B, 16, T, 128), "TFLOP/s"
     elif args.workload == "profile_decode":
         q, r, kc, vc, sl = inputs.decode_inputs(16, 16, 8192, 128, seed=2)
         q, r, kc, vc = (t.torch().to(dev) for t in (q, r, kc, vc))
@@ -564,7 +566,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["default", "prefill_long", "sweep", "profile_fwd", "profile_decode",
-                                           "profile_rho", "profile_paged"], default="default")
+                                           "profile_rho", "profile_paged", "profile_fwd_long"], default="default")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
