@@ -70,10 +70,6 @@ template <> __device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat
     *p = __float2bfloat16_rn(v);
 }
 
-// Minimum page size of the paged layout; a sub-chunk then spans at most
-// SUB / MIN_PAGE + 2 pages.
-constexpr int MIN_PAGE = 16;
-
 template <int D> struct DecodeSmem {
     static constexpr int LPT = D / 8;        // lanes per token row
     static constexpr int TPW = 32 / LPT;     // token rows per warp step
@@ -83,18 +79,13 @@ template <int D> struct DecodeSmem {
     float red_o[GROUPS][D];
     float red_m[GROUPS][D];
     float red_s[3][NW];
-    int page[SUB / MIN_PAGE + 2];            // paged layout: page ids of the current sub-chunk
 };
 
-// PAGED: kc, vc are [num_pages, Hkv, page_size, d]; token t of sequence b sits
-// in page table[b * max_pages + t / page_size], row t % page_size, and query
-// head h reads KV head h / group.  Unpaged: kc, vc are [B, H, Tcap, d].
-template <int D, typename Tout, bool PAGED>
+template <int D, typename Tout>
 __global__ void __launch_bounds__(NTHREADS, MIN_BLOCKS) k_decode_split(
     const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ rho, const __nv_bfloat16 *__restrict__ kc,
     const __nv_bfloat16 *__restrict__ vc, const int *__restrict__ seqlens, Tout *__restrict__ y,
-    float *__restrict__ lse, int H, int Tcap, int chunk, int nsplit, long BH, float *__restrict__ partials,
-    PagedKV pg, int *__restrict__ err) {
+    float *__restrict__ lse, int H, int Tcap, int chunk, int nsplit, long BH, float *__restrict__ partials) {
     using S = DecodeSmem<D>;
     constexpr int LPT = S::LPT, TPW = S::TPW, GROUPS = S::GROUPS;
     constexpr int STEP = GROUPS * UNROLL;    // token rows per unrolled step
@@ -123,12 +114,8 @@ __global__ void __launch_bounds__(NTHREADS, MIN_BLOCKS) k_decode_split(
             unpack8(__ldg(qp), qv);
             unpack8(__ldg(rp), rv);
         }
-        // unpaged: the head's rows; paged: the KV head's rows within a page
-        const size_t head_off = PAGED ? (size_t)((int)(bh % H) / pg.group) * ((size_t)1 << pg.pshift) * D
-                                      : (size_t)bh * Tcap * D;
-        const uint4 *kbase = reinterpret_cast<const uint4 *>(kc + head_off) + c;
-        const uint4 *vbase = reinterpret_cast<const uint4 *>(vc + head_off) + c;
-        const size_t page_stride = PAGED ? (size_t)pg.Hkv * ((size_t)1 << pg.pshift) * LPT : 0;   // in uint4
+        const uint4 *kbase = reinterpret_cast<const uint4 *>(kc + (size_t)bh * Tcap * D) + c;
+        const uint4 *vbase = reinterpret_cast<const uint4 *>(vc + (size_t)bh * Tcap * D) + c;
 
         float mu = -INFINITY, lsum = 0.f, asum = 0.f;
         float O[8], M[8];
@@ -137,43 +124,13 @@ __global__ void __launch_bounds__(NTHREADS, MIN_BLOCKS) k_decode_split(
 
         for (int s0 = t0; s0 < t1; s0 += SUB) {
             const int n = min(SUB, t1 - s0);
-            int p0 = 0;
-            if constexpr (PAGED) {
-                // page ids of this sub-chunk, checked against the page count
-                p0 = s0 >> pg.pshift;
-                const int np = ((s0 + n - 1) >> pg.pshift) - p0 + 1;
-                for (int i = tid; i < np; i += NTHREADS) {
-                    int id = pg.table[(size_t)b * pg.max_pages + p0 + i];
-                    if (id < 0 || id >= pg.num_pages) {
-                        atomicExch(err, PARALLAX_ERR_DEVICE_INDEX);
-                        id = -1;
-                    }
-                    sm.page[i] = id;
-                }
-                __syncthreads();
-            }
-            // address of token t's row (nullptr for a rejected page id)
-            auto row = [&](const uint4 *base, int t) -> const uint4 * {
-                if constexpr (PAGED) {
-                    const int id = sm.page[(t >> pg.pshift) - p0];
-                    if (id < 0) return nullptr;
-                    return base + (size_t)id * page_stride + (size_t)(t & ((1 << pg.pshift) - 1)) * LPT;
-                } else {
-                    return base + (size_t)t * LPT;
-                }
-            };
             // ---- pass A: K stream -> z (log2 units) and a ----
             for (int base = 0; base < n; base += STEP) {
                 uint4 kr[UNROLL];
 #pragma unroll
                 for (int x = 0; x < UNROLL; ++x) {
                     const int tok = base + x * GROUPS + slot;
-                    if constexpr (PAGED) {
-                        const uint4 *pk = tok < n ? row(kbase, s0 + tok) : nullptr;
-                        kr[x] = pk ? ldg_stream(pk) : make_uint4(0, 0, 0, 0);
-                    } else {
-                        kr[x] = tok < n ? ldg_stream(kbase + (size_t)(s0 + tok) * LPT) : make_uint4(0, 0, 0, 0);
-                    }
+                    kr[x] = tok < n ? ldg_stream(kbase + (size_t)(s0 + tok) * LPT) : make_uint4(0, 0, 0, 0);
                 }
 #pragma unroll
                 for (int x = 0; x < UNROLL; ++x) {
@@ -233,12 +190,7 @@ __global__ void __launch_bounds__(NTHREADS, MIN_BLOCKS) k_decode_split(
 #pragma unroll
                 for (int x = 0; x < UNROLL; ++x) {
                     const int tok = base + x * GROUPS + slot;
-                    if constexpr (PAGED) {
-                        const uint4 *pv = tok < n ? row(vbase, s0 + tok) : nullptr;
-                        vr[x] = pv ? ldg_stream(pv) : make_uint4(0, 0, 0, 0);
-                    } else {
-                        vr[x] = tok < n ? ldg_stream(vbase + (size_t)(s0 + tok) * LPT) : make_uint4(0, 0, 0, 0);
-                    }
+                    vr[x] = tok < n ? ldg_stream(vbase + (size_t)(s0 + tok) * LPT) : make_uint4(0, 0, 0, 0);
                 }
 #pragma unroll
                 for (int x = 0; x < UNROLL; ++x) {
@@ -426,34 +378,18 @@ cudaError_t launch_combine(const float *partials, const int *seqlens, void *y, f
     return cudaGetLastError();
 }
 
-template <int D, typename Tout, bool PAGED>
+template <int D, typename Tout>
 cudaError_t launch_t(const void *q, const void *rho, const void *kc, const void *vc, const int *seqlens, void *y,
-                     float *lse, int B, int H, int Tcap, const DecodePlan &p, float *partials, const PagedKV &pg,
-                     int *err, cudaStream_t s) {
+                     float *lse, int B, int H, int Tcap, const DecodePlan &p, float *partials, cudaStream_t s) {
     const long BH = (long)B * H;
     const long units = BH * p.nsplit;
     const long grid = units < 0x7fffffffL ? units : 0x7fffffffL;   // one CTA per unit
-    k_decode_split<D, Tout, PAGED><<<(unsigned)grid, NTHREADS, 0, s>>>(
+    k_decode_split<D, Tout><<<(unsigned)grid, NTHREADS, 0, s>>>(
         (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)rho, (const __nv_bfloat16 *)kc, (const __nv_bfloat16 *)vc,
-        seqlens, (Tout *)y, lse, H, Tcap, p.chunk, p.nsplit, BH, partials, pg, err);
+        seqlens, (Tout *)y, lse, H, Tcap, p.chunk, p.nsplit, BH, partials);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || p.nsplit == 1) return e;
     return launch_combine<D, Tout>(partials, seqlens, y, lse, B, H, p, s);
-}
-
-template <bool PAGED>
-cudaError_t launch_any(const void *q, const void *rho, const void *kc, const void *vc, const int *seqlens, void *y,
-                       float *lse, int B, int H, int Tcap, int d, int out_dtype, const DecodePlan &p, float *partials,
-                       const PagedKV &pg, int *err, cudaStream_t s) {
-    if (d == 64) {
-        if (out_dtype == PARALLAX_F32)
-            return launch_t<64, float, PAGED>(q, rho, kc, vc, seqlens, y, lse, B, H, Tcap, p, partials, pg, err, s);
-        return launch_t<64, __nv_bfloat16, PAGED>(q, rho, kc, vc, seqlens, y, lse, B, H, Tcap, p, partials, pg, err,
-                                                  s);
-    }
-    if (out_dtype == PARALLAX_F32)
-        return launch_t<128, float, PAGED>(q, rho, kc, vc, seqlens, y, lse, B, H, Tcap, p, partials, pg, err, s);
-    return launch_t<128, __nv_bfloat16, PAGED>(q, rho, kc, vc, seqlens, y, lse, B, H, Tcap, p, partials, pg, err, s);
 }
 
 }  // namespace
@@ -484,29 +420,30 @@ size_t decode_partials_bytes(int B, int H, int d, const DecodePlan &p) {
 cudaError_t launch_decode(const void *q, const void *rho, const void *kc, const void *vc, const int *seqlens,
                           void *y, float *lse, int B, int H, int Tcap, int d, int out_dtype, const DecodePlan &p,
                           float *partials, int sm_count, const DeviceCtl &ctl, cudaStream_t s) {
+    (void)ctl;   // this kernel has no device-side waits
     (void)sm_count;
-    const PagedKV none{nullptr, 0, 0, 0, 1, 1};
-    return launch_any<false>(q, rho, kc, vc, seqlens, y, lse, B, H, Tcap, d, out_dtype, p, partials, none, ctl.err,
-                             s);
+    if (d == 64) {
+        if (out_dtype == PARALLAX_F32)
+            return launch_t<64, float>(q, rho, kc, vc, seqlens, y, lse, B, H, Tcap, p, partials, s);
+        return launch_t<64, __nv_bfloat16>(q, rho, kc, vc, seqlens, y, lse, B, H, Tcap, p, partials, s);
+    }
+    if (out_dtype == PARALLAX_F32)
+        return launch_t<128, float>(q, rho, kc, vc, seqlens, y, lse, B, H, Tcap, p, partials, s);
+    return launch_t<128, __nv_bfloat16>(q, rho, kc, vc, seqlens, y, lse, B, H, Tcap, p, partials, s);
 }
 
 DecodePlan plan_decode_paged(int B, int Hq, int Hkv, int Tcap, int d, int sm_count) {
+    // a 4-warp tensor-core unit serves up to 8 query heads of a KV head; it is
+    // sized like four split-kernel units so that each warp streams enough
+    // tiles to amortise its pipeline fill and the final merge
     const int group = Hq / Hkv;
-    // grouped heads: a 4-warp tensor-core unit serves up to 8 query heads of a
-    // KV head; it is sized like four split-kernel units so that each warp
-    // streams enough tiles to amortise its pipeline fill and the final merge
-    if (group >= 2) return plan_decode(B, Hkv * ((group + 7) / 8) * 4, Tcap, d, sm_count);
-    return plan_decode(B, Hq, Tcap, d, sm_count);
+    return plan_decode(B, Hkv * ((group + 7) / 8) * 4, Tcap, d, sm_count);
 }
 
 cudaError_t launch_decode_paged(const void *q, const void *rho, const void *kpages, const void *vpages,
                                 const PagedKV &pg, const int *seqlens, void *y, float *lse, int B, int Hq, int d,
                                 int out_dtype, const DecodePlan &p, float *partials, const DeviceCtl &ctl,
                                 cudaStream_t s) {
-    const int Tcap = pg.max_pages << pg.pshift;
-    if (pg.group < 2)
-        return launch_any<true>(q, rho, kpages, vpages, seqlens, y, lse, B, Hq, Tcap, d, out_dtype, p, partials, pg,
-                                ctl.err, s);
     cudaError_t e = launch_decode_gqa_split(q, rho, kpages, vpages, pg, seqlens, y, lse, B, Hq, d, out_dtype, p,
                                             partials, ctl.err, s);
     if (e != cudaSuccess || p.nsplit == 1) return e;

@@ -44,7 +44,7 @@ struct PagedKV {
 };
 // Split plan of the paged decode for the kernel that serves this head grouping.
 DecodePlan plan_decode_paged(int B, int Hq, int Hkv, int Tcap, int d, int sm_count);
-// Tensor-core split kernel for grouped heads (Hq / Hkv >= 2); writes the same
+// Tensor-core split kernel of the paged decode (any Hq / Hkv); writes the same
 // partials (or y when nsplit == 1) as the split decode kernel.
 cudaError_t launch_decode_gqa_split(const void *q, const void *rho, const void *kpages, const void *vpages,
                                     const PagedKV &pg, const int *seqlens, void *y, float *lse, int B, int Hq, int d,

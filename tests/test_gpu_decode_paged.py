@@ -45,9 +45,10 @@ def test_paged_grouped_small(group, page_size, d):
     parity.assert_lse(lg[1:], lr[1:])
 
 
-def test_paged_identity_table_equals_contiguous_decode_bitwise():
+def test_paged_identity_table_matches_contiguous_decode():
     """A contiguous cache cut into pages in order, one query head per KV head:
-    the paged call reproduces parallax_decode bit for bit (same split plan)."""
+    the paged call (tensor-core kernel) agrees with parallax_decode (CUDA-core
+    split kernel) within the bf16 gate, and both with the oracle."""
     B, H, ps, max_pages, d = 6, 4, 64, 40, 128
     tcap = ps * max_pages
     sl = inputs.ragged_seqlens(B, tcap, 9)
@@ -61,7 +62,10 @@ def test_paged_identity_table_equals_contiguous_decode_bitwise():
     kp, vp = pages(kc.torch().to(DEV)), pages(vc.torch().to(DEV))
     table = torch.arange(B * max_pages, dtype=torch.int32, device=DEV).reshape(B, max_pages)
     y, lse = _run((q.torch().to(DEV), rho.torch().to(DEV), kp, vp, table, torch.from_numpy(sl).to(DEV)))
-    assert torch.equal(y, y_ref) and torch.equal(lse, l_ref)
+    parity.assert_bf16_parity(y.cpu().numpy(), y_ref.cpu().numpy(), 2, "paged vs contiguous")
+    parity.assert_lse(lse.cpu().numpy(), l_ref.cpu().numpy())
+    yr, _ = oracle.decode(q.f64, rho.f64, kc.f64, vc.f64, sl)
+    parity.assert_bf16_parity(y.cpu().numpy(), yr, 2, "paged vs oracle")
 
 
 def test_bad_page_id_is_reported_and_unreached_entries_are_ignored():
