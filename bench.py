@@ -529,6 +529,15 @@ def oracle_sample(budget_s=12.0):
     dt = (time.perf_counter() - t0) / reps
     dec_tbs = decode_bytes(nbs, dc["H"], dc["d"], sl) / dt / 1e12
     dec_sample = f"{nbs * dc['H']} of the {dc['B'] * dc['H']} heads x {dc['Tcap']} tokens, x{reps}"
+    # the same oracle on one thread, on the first sequence (16 heads)
+    oracle.set_threads(1)
+    try:
+        t0 = time.perf_counter()
+        oracle.decode(qf[:1], rf[:1], kf[:1], vf[:1], sl[:1])
+        dt1 = time.perf_counter() - t0
+    finally:
+        oracle.set_threads(cores)
+    dec_tbs_1t = decode_bytes(1, dc["H"], dc["d"], sl[:1]) / dt1 / 1e12
 
     pc = PREFILL_CFG
     pq, pk, pv, pr = inputs.fwd_bf16_inputs(1, 1, pc["T"], pc["d"], seed=3)
@@ -539,20 +548,21 @@ def oracle_sample(budget_s=12.0):
     pairs = int(np.sum(rows + 1))
     pre_tfs = 8 * pc["d"] * pairs / dt / 1e12
     pre_sample = f"{rows.size} causal rows (every 8th) of one T={pc['T']} head, {pairs} pairs"
-    return cores, dec_tbs, dec_sample, pre_tfs, pre_sample
+    return cores, dec_tbs, dec_sample, pre_tfs, pre_sample, dec_tbs_1t
 
 
 def run_reference(args, rank, world):
     if rank != 0:
         return None
-    cores, dec_tbs, dec_sample, pre_tfs, pre_sample = oracle_sample()
+    cores, dec_tbs, dec_sample, pre_tfs, pre_sample, dec_1t = oracle_sample()
     line = {
         "metric": METRIC, "value": dec_tbs, "unit": "TB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
         "config": {"workload": "decode step B=64 H=16 d=128 ctx=4096 (headline) + prefill B=8 T=4096 H=16 d=128",
                    "decode": dict(DECODE_CFG), "prefill": dict(PREFILL_CFG)},
-        "cpu_baseline": {"value": dec_tbs, "unit": "TB/s", "cores": cores, "kind": "oracle", "sample": dec_sample},
+        "cpu_baseline": {"value": dec_tbs, "unit": "TB/s", "cores": cores, "kind": "oracle", "sample": dec_sample,
+                         "value_1_thread": dec_1t},
         "prefill": {"value": pre_tfs, "unit": "TFLOP/s", "sample": pre_sample},
         "e2e": {"value": dec_tbs, "unit": "TB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -594,9 +604,9 @@ def main():
     else:
         line = run_ours(args, rank, world)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
-            cores, dec_tbs, dec_sample, _, _ = oracle_sample(budget_s=10.0)
+            cores, dec_tbs, dec_sample, _, _, dec_1t = oracle_sample(budget_s=10.0)
             line["cpu_baseline"] = {"value": dec_tbs, "unit": "TB/s", "cores": cores, "kind": "oracle",
-                                    "sample": dec_sample}
+                                    "sample": dec_sample, "value_1_thread": dec_1t}
     if rank == 0 and line is not None:
         print(json.dumps(line), flush=True)
     if world > 1 and args.impl == "ours":
