@@ -152,9 +152,9 @@ PARALLAX_API int parallax_decode_ex(const void *q, const void *rho, const void *
  *   y              : [B, Hq, d] of out_dtype (F32 or BF16); lse [B, Hq] fp32 or NULL.
  *   B, Hkv >= 1; Hq a multiple of Hkv; page_size a power of two in [16, 4096];
  *   max_pages, num_pages >= 1; d in {64, 128}; in_dtype BF16.
- * Split partials use the library's scratch, sized as
- * parallax_decode_workspace_bytes(B, Hq, max_pages * page_size, d).  Calls
- * sharing the library's scratch must be ordered on the device.
+ * Split partials use the library's scratch, which grows on demand (a
+ * cudaMalloc, after a device synchronization, the first time a shape needs
+ * more).  Calls sharing the library's scratch must be ordered on the device.
  */
 PARALLAX_API int parallax_decode_paged(const void *q, const void *rho, const void *kpages, const void *vpages,
                                        const int *block_table, const int *seqlens, void *y, float *lse, int B,
