@@ -348,12 +348,8 @@ cudaError_t launch_t(const void *q, const void *rho, const void *kpages, const v
                      const int *seqlens, void *y, float *lse, int B, int Hq, const DecodePlan &p, float *partials,
                      int *err, cudaStream_t s) {
     constexpr int SMEM = GqaSmem<D>::BYTES;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(k_decode_gqa<D, Tout>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static std::atomic<unsigned long long> limit_set{0};
+    if (cudaError_t e = ensure_smem_limit(k_decode_gqa<D, Tout>, SMEM, limit_set)) return e;
     const int htiles = (pg.group + 7) / 8;
     const long per_split = (long)B * pg.Hkv * htiles;
     const long units = per_split * p.nsplit;

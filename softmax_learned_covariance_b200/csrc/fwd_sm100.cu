@@ -619,13 +619,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 template <bool WITH_RHO, typename Tout>
 cudaError_t launch_t(const FwdTensorMaps &tm, void *y, float *lse, int BH, int T, int causal, int sm_count,
                      int *work_counter, const DeviceCtl &ctl, cudaStream_t s) {
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(k_fwd<WITH_RHO, Tout>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static std::atomic<unsigned long long> limit_set{0};
+    if (cudaError_t e = ensure_smem_limit(k_fwd<WITH_RHO, Tout>, (int)SMEM_BYTES, limit_set)) return e;
     const int items = ((T + BM - 1) / BM) * BH;
     const int grid = items < sm_count ? items : sm_count;
     cudaError_t e = cudaMemsetAsync(work_counter, 0, sizeof(int), s);

@@ -1,5 +1,6 @@
 // internal.h -- launch entry points shared between the host API and the kernels.
 #pragma once
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 #include <cuda.h>
@@ -8,6 +9,20 @@
 #include "parallax.h"
 
 namespace plx {
+
+// Raises kernel `f`'s dynamic shared-memory limit to `bytes` once per device
+// (function attributes belong to a device's context; `done` remembers the
+// devices already set, for device ordinals below 64).
+template <typename F> cudaError_t ensure_smem_limit(F f, int bytes, std::atomic<unsigned long long> &done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = dev < 64 ? 1ull << dev : 0ull;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
+    return e;
+}
 
 // Per-launch wait policy: absolute %globaltimer deadline is computed in-kernel
 // from this budget (nanoseconds).

@@ -175,12 +175,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
 cudaError_t launch_rho_proj(const CUtensorMap &tm_x, const CUtensorMap &tm_w, void *rho, int B, int T, int d_model,
                             int H, int d, int sm_count, const DeviceCtl &ctl, cudaStream_t s) {
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(k_rho_proj, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static std::atomic<unsigned long long> limit_set{0};
+    if (cudaError_t e = ensure_smem_limit(k_rho_proj, (int)SMEM_BYTES, limit_set)) return e;
     const int M = B * T, N = H * d;
     const int tiles = ((M + BM - 1) / BM) * (N / BN);
     const int grid = tiles < sm_count ? tiles : sm_count;
