@@ -12,6 +12,9 @@ library is missing or a call fails, a ``ParallaxError`` is raised.
 Functions keep the C names:
     parallax_fwd(q, k, v, rho=None, causal=True, out_dtype=torch.float32) -> (y, lse)
     parallax_decode(q, rho, kcache, vcache, seqlens, out_dtype=torch.float32) -> (y, lse)
+    parallax_decode_ex(..., workspace) -> (y, lse)          caller-owned split scratch
+    parallax_decode_paged(q, rho, kpages, vpages, block_table, seqlens) -> (y, lse)
+                                                            paged cache, grouped query heads
     parallax_rho_proj(x, W_R, H, d) -> rho
 """
 from __future__ import annotations
