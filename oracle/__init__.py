@@ -19,6 +19,9 @@ Parity status of each function (how it is pinned, see ``tests/test_oracle_pins.p
   decode_paged            : pinned to decode, a layout change only (identity page
                             table on a contiguous cache, permuted pages, grouped
                             heads equal to replicated key/value heads)
+  bwd / rho_proj_bwd      : pinned (central finite differences of the forward
+                            oracle; at rho = 0, autograd of library SDPA; autograd
+                            of a library matmul); no CUDA counterpart yet
 """
 from __future__ import annotations
 
@@ -174,6 +177,64 @@ class Oracle:
         if rc:
             raise ValueError(f"oracle_rho_proj rejected its arguments (code {rc})")
         return out
+
+
+def bwd(q, k, v, rho, dy, causal: bool = True):
+    """Gradients of the Parallax forward: (dq, dk, dv, drho) for an upstream dy.
+
+    The operator per head (zubnet.ai news item on Parallax, paragraph 2; the
+    forward this module computes): Z = Q K^T / sqrt(d) (keys past the query
+    masked when causal), S = softmax over keys, A = R K^T, abar = rowsum(S o A),
+    O = S V, M = (S o A) V, Y = O - M + abar * O.  The pages train with this
+    operator but print no backward; what follows is the chain rule through
+    those definitions, in that order, for L = <dY, Y>:
+        dO    = dY (1 + abar)            dabar = rowsum(dY o O)      dM = -dY
+        dV    = S^T dO + (S o A)^T dM
+        dS    = (dY V^T) o (1 + abar - A) + dabar o A
+        dA    = S o (dabar - dY V^T)
+        dZ    = S o (dS - rowsum(S o dS))           (softmax backward)
+        dQ    = dZ K / sqrt(d)    dK = dZ^T Q / sqrt(d) + dA^T R    dR = dA K
+    Plain fp64 numpy, one head at a time, no blocking.  q, k, v, rho, dy: [B, H, T, d].
+    """
+    q, k, v, rho, dy = (np.asarray(t, np.float64) for t in (q, k, v, rho, dy))
+    B, H, T, d = q.shape
+    out = [np.zeros_like(q) for _ in range(4)]
+    mask = np.tril(np.ones((T, T), bool)) if causal else np.ones((T, T), bool)
+    sc = 1.0 / np.sqrt(d)
+    for b in range(B):
+        for h in range(H):
+            Q, K, V, R, dY = q[b, h], k[b, h], v[b, h], rho[b, h], dy[b, h]
+            Z = np.where(mask, (Q @ K.T) * sc, -np.inf)
+            S = np.exp(Z - Z.max(axis=1, keepdims=True))
+            S = S / S.sum(axis=1, keepdims=True)
+            A = R @ K.T
+            abar = (S * A).sum(axis=1, keepdims=True)
+            O = S @ V
+            dO = dY * (1.0 + abar)
+            dabar = (dY * O).sum(axis=1, keepdims=True)
+            dM = -dY
+            dV = S.T @ dO + (S * A).T @ dM
+            G = dY @ V.T
+            dS = G * (1.0 + abar - A) + dabar * A
+            dA = S * (dabar - G)
+            dZ = S * (dS - (S * dS).sum(axis=1, keepdims=True))
+            out[0][b, h] = dZ @ K * sc
+            out[1][b, h] = dZ.T @ Q * sc + dA.T @ R
+            out[2][b, h] = dV
+            out[3][b, h] = dA @ K
+    return tuple(out)
+
+
+def rho_proj_bwd(x, W_R, drho, H: int, d: int):
+    """Gradients of rho[b, h, t, :] = x[b, t, :] W_R[:, h d:(h+1) d] for an upstream drho:
+    dx = drho' W_R^T and dW_R = sum over (b, t) of x^T drho', with drho' the
+    [B, T, H d] regrouping of drho.  fp64."""
+    x, W, g = np.asarray(x, np.float64), np.asarray(W_R, np.float64), np.asarray(drho, np.float64)
+    B, T, dm = x.shape
+    g2 = g.transpose(0, 2, 1, 3).reshape(B, T, H * d)
+    dx = g2 @ W.T
+    dW = np.einsum("btc,btn->cn", x, g2)
+    return dx, dW
 
 
 def _f64(a):
