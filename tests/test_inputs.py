@@ -34,3 +34,18 @@ def test_sweep_grid_skips_cells_over_120GB():
     assert len(cells) == 30
     skipped = [(b, c) for _, b, c, _, s in cells if s]
     assert sorted(skipped) == [(1024, 32768), (2048, 8192), (2048, 32768)]
+
+
+def test_paged_decode_inputs_shapes_and_table():
+    sl = np.array([100, 0, 64], np.int32)
+    q, rho, kp, vp, table, sl2 = inputs.paged_decode_inputs(3, 8, 2, 32, 5, 64, sl, seed=1, spare_pages=4)
+    assert q.bits.shape == (3, 8, 64) and rho.bits.shape == (3, 8, 64)
+    assert kp.bits.shape == vp.bits.shape == (3 * 5 + 4, 2, 32, 64)
+    assert table.shape == (3, 5) and table.dtype == np.int32
+    # distinct page ids drawn from the pool: every sequence's pages are its own
+    flat = table.reshape(-1)
+    assert len(set(flat.tolist())) == flat.size and flat.min() >= 0 and flat.max() < 3 * 5 + 4
+    assert np.array_equal(sl2, sl)
+    # deterministic in the seed
+    again = inputs.paged_decode_inputs(3, 8, 2, 32, 5, 64, sl, seed=1, spare_pages=4)
+    assert np.array_equal(again[4], table) and np.array_equal(again[2].bits, kp.bits)
