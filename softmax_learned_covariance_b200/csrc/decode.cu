@@ -28,9 +28,10 @@ namespace plx {
 namespace {
 
 // Measured on B200 (bench shape B=64 H=16 ctx 4096): 2-warp CTAs with 16 of them
-// resident per SM (64 registers per thread) stream at 5.50 TB/s, 4-warp CTAs at
-// 8 per SM at 5.26 TB/s, 8-warp CTAs at 3 per SM at 4.5 TB/s, and a TMA-ring
-// variant whose consumer warps were latency bound per block at 3.6-3.8 TB/s.
+// resident per SM (64 registers per thread) stream at 5.3-5.5 TB/s across runs,
+// 4-warp CTAs at 8 per SM at 5.1-5.26 TB/s, 8-warp CTAs at 3 per SM at 4.4-4.5
+// TB/s, and a TMA-ring variant whose consumer warps were latency bound per block
+// at 3.6-3.8 TB/s.
 // Small CTAs keep the __syncthreads-separated phases of one CTA from idling the
 // SM: the other CTAs' loads are in flight meanwhile.
 constexpr int NW = 2;            // warps per CTA

@@ -42,8 +42,8 @@ cudaError_t launch_fwd_simt(const void *q, const void *k, const void *v, const v
 
 // split-KV decode + combine
 struct DecodePlan {
-    int nsplit;      // CTAs per (b,h)
-    int chunk;       // tokens per split (multiple of 64)
+    int nsplit;      // chunks per sequence (units per head)
+    int chunk;       // tokens per chunk: a multiple of 128, or the whole cache
 };
 DecodePlan plan_decode(int B, int H, int Tcap, int d, int sm_count);
 size_t decode_partials_bytes(int B, int H, int d, const DecodePlan &p);
