@@ -27,7 +27,9 @@
  *     prints, never aborts and never falls back to another implementation.
  *   - Device-side waits are bounded.  A wait that gives up records
  *     PARALLAX_ERR_DEVICE_TIMEOUT in a per-device error word and the kernel
- *     returns; read it with parallax_last_device_error().
+ *     returns; an out-of-range page id met by the paged decode records
+ *     PARALLAX_ERR_DEVICE_INDEX there.  Read (and clear) it with
+ *     parallax_last_device_error().
  *   - The library keeps one grow-only scratch allocation per device (the fp16
  *     copy of V for the prefill kernel, the split partials for decode).  It
  *     grows with cudaMalloc on first use, so the first call at a new, larger
