@@ -547,7 +547,7 @@ def oracle_sample(budget_s=12.0):
     dt = time.perf_counter() - t0
     pairs = int(np.sum(rows + 1))
     pre_tfs = 8 * pc["d"] * pairs / dt / 1e12
-    pre_sample = f"{rows.size} causal rows (every 8th) of one T={pc['T']} head, {pairs} pairs"
+    pre_sample = f"{rows.size} causal rows (every 8th) of one T={pc['T']} head, {pairs} pairs, {pairs / dt:.3e} pairs/s"
     return cores, dec_tbs, dec_sample, pre_tfs, pre_sample, dec_tbs_1t
 
 
