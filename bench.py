@@ -26,6 +26,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -109,12 +110,12 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        self.path = None
 
     def start(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.f = open(self.path, "w")
+            fd, self.path = tempfile.mkstemp(prefix=f"parallax_clocks_{self.gpu}_", suffix=".csv")
+            self.f = os.fdopen(fd, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                  "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
@@ -144,6 +145,10 @@ class ClockSampler:
             for n, v in zip(names, parts[5:9]):
                 if v.lower() == "active":
                     reasons.add(n)
+        try:
+            os.unlink(self.path)
+        except OSError:
+            pass
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
@@ -219,11 +224,48 @@ def run_profile_case(args):
     return {"workload": args.workload, "ms": ms, "value": work / (ms * 1e-3) / 1e12, "unit": unit}
 
 
+def time_decode_cell(plx, torch, dev, b, ctx, idx, steps, warmup, flush, peak):
+    """One decode sweep cell: H=16, d=128, batch b, context ctx, ragged lengths in
+    [ctx/2, ctx] (seeded by the cell index), inputs drawn on the device.  Cells
+    whose cache could stay in L2 are timed call by call with a 256 MB write
+    between calls; the others stream past L2 anyway."""
+    from softmax_learned_covariance_b200 import inputs
+
+    sl = inputs.ragged_seqlens(b, ctx, 4 + idx)
+    q, r, kc, vc, dsl = inputs.decode_inputs_device(b, 16, ctx, 128, sl, seed=4 + idx, device=dev)
+    y = torch.empty((b, 16, 128), dtype=torch.float32, device=dev)
+    for _ in range(warmup):
+        plx.parallax_decode(q, r, kc, vc, dsl, y=y, want_lse=False)
+    torch.cuda.synchronize()
+    nbytes = 2 * b * 16 * ctx * 128 * 2
+    small = nbytes < (256 << 20)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps if small else 1)]
+    if small:
+        for a, e in ev:
+            flush.fill_(1)
+            a.record()
+            plx.parallax_decode(q, r, kc, vc, dsl, y=y, want_lse=False)
+            e.record()
+    else:
+        ev[0][0].record()
+        for _ in range(steps):
+            plx.parallax_decode(q, r, kc, vc, dsl, y=y, want_lse=False)
+        ev[0][1].record()
+    torch.cuda.synchronize()
+    assert plx.parallax_last_device_error() == 0
+    ms = sum(a.elapsed_time(e) for a, e in ev) / steps
+    nb = decode_bytes(b, 16, 128, sl)
+    gbs = nb / (ms * 1e-3) / 1e9
+    del q, r, kc, vc, dsl, y
+    torch.cuda.empty_cache()
+    return {"B": b, "ctx": ctx, "ms": round(ms, 4), "GB/s": round(gbs, 1), "frac": round(gbs / peak, 4),
+            "bytes": nb, "l2_flushed": small, "long_context": bool(ctx >= 8192 and b * 16 >= 128)}
+
+
 def run_sweep(args):
     """Decode sweep: heads 16, d 128, batch x context grid with ragged lengths in
-    [ctx/2, ctx]; cells whose cache exceeds 120 GB are skipped.  Inputs are drawn
-    on the device (seeded); cells small enough to sit in L2 are timed with an
-    L2 flush before every call."""
+    [ctx/2, ctx]; cells whose cache exceeds 120 GB are skipped."""
     import torch
 
     import softmax_learned_covariance_b200 as plx
@@ -238,43 +280,37 @@ def run_sweep(args):
         if skipped:
             cells.append({"B": b, "ctx": ctx, "skipped": "cache %.0f GB > 120 GB" % (nbytes / 1e9)})
             continue
-        sl = inputs.ragged_seqlens(b, ctx, 4 + idx)
-        q, r, kc, vc, dsl = inputs.decode_inputs_device(b, 16, ctx, 128, sl, seed=4 + idx, device=dev)
-        y = torch.empty((b, 16, 128), dtype=torch.float32, device=dev)
-        for _ in range(args.warmup):
-            plx.parallax_decode(q, r, kc, vc, dsl, y=y, want_lse=False)
-        torch.cuda.synchronize()
-        # Cells whose cache would stay in the 126 MB L2 are timed call by call
-        # with a 256 MB write between calls; the others stream past L2 anyway.
-        small = nbytes < (256 << 20)
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps if small else 1)]
-        if small:
-            for a, e in ev:
-                flush.fill_(1)
-                a.record()
-                plx.parallax_decode(q, r, kc, vc, dsl, y=y, want_lse=False)
-                e.record()
-        else:
-            ev[0][0].record()
-            for _ in range(args.steps):
-                plx.parallax_decode(q, r, kc, vc, dsl, y=y, want_lse=False)
-            ev[0][1].record()
-        torch.cuda.synchronize()
-        assert plx.parallax_last_device_error() == 0
-        ms = sum(a.elapsed_time(e) for a, e in ev) / args.steps
-        nb = decode_bytes(b, 16, 128, sl)
-        gbs = nb / (ms * 1e-3) / 1e9
-        cells.append({"B": b, "ctx": ctx, "ms": round(ms, 4), "GB/s": round(gbs, 1),
-                      "frac": round(gbs / peaks["hbm_gbs"], 4), "bytes": nb, "l2_flushed": small,
-                      "long_context": bool(ctx >= 8192 and b * 16 >= 128)})
-        del q, r, kc, vc, dsl, y
-        torch.cuda.empty_cache()
+        cells.append(time_decode_cell(plx, torch, dev, b, ctx, idx, args.steps, args.warmup, flush,
+                                      peaks["hbm_gbs"]))
     longc = [c["frac"] for c in cells if c.get("long_context")]
     return {"workload": "decode sweep H=16 d=128, ragged lengths in [ctx/2, ctx]", "unit": "GB/s",
             "steps": args.steps, "warmup": args.warmup,
             "peak": peaks["hbm_gbs"], "peak_note": "measured HBM copy bandwidth" if peaks["source"] == "measured"
             else "fallback", "long_context_min_frac": min(longc) if longc else None, "cells": cells}
+
+
+# Long-context cells of the decode sweep measured in the default line (ctx >= 8192
+# with B*H >= 128, where the sweep's >= 70 % of HBM gate applies); the larger
+# ones (up to 69 GB of cache) are left to --workload sweep.
+DECODE_LONG_CELLS = ((8, 8192), (8, 32768), (64, 8192), (256, 8192))
+
+
+def measure_decode_long(args, peaks):
+    import torch
+
+    import softmax_learned_covariance_b200 as plx
+    from softmax_learned_covariance_b200 import inputs
+
+    dev = torch.cuda.current_device()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    index = {(b, c): i for i, b, c, _, _ in inputs.sweep_cells()}
+    cells = [time_decode_cell(plx, torch, dev, b, c, index[(b, c)], args.steps, args.warmup, flush,
+                              peaks["hbm_gbs"]) for b, c in DECODE_LONG_CELLS]
+    del flush
+    torch.cuda.empty_cache()
+    return {"workload": "decode sweep long-context cells, H=16 d=128, ragged lengths in [ctx/2, ctx]",
+            "unit": "GB/s", "peak": peaks["hbm_gbs"], "gate": 0.70,
+            "min_frac": min(c["frac"] for c in cells), "cells": cells}
 
 
 def run_ours(args, rank, world):
@@ -392,6 +428,7 @@ def run_ours(args, rank, world):
                    "h2d_bytes_per_step": h2d_p, "d2h_bytes_per_step": yp.numel() * 4, "steps": ksteps}
 
     extras = measure_extras(args, stream, barrier, world, peaks, pc, dpq, dpk, dpv, yp, lp, fwd_ms)
+    decode_long = None if args.no_decode_long else measure_decode_long(args, peaks)
 
     dec_tbs = whole_job_rate(d_bytes, dec_ms, world) / 1e12
     fwd_tfs = whole_job_rate(p_flops, fwd_ms, world) / 1e12
@@ -433,6 +470,7 @@ def run_ours(args, rank, world):
         "e2e": e2e,
         "decode_paged": extras["decode_paged"],
         "softmax_only_fwd": extras["softmax_only_fwd"],
+        "decode_long": decode_long,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
         "peaks": peaks,
@@ -579,6 +617,7 @@ def main():
                                            "profile_rho", "profile_paged", "profile_fwd_long"], default="default")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode-long", action="store_true", help="skip the long-context decode cells")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -30,10 +30,17 @@
  *     returns; an out-of-range page id met by the paged decode records
  *     PARALLAX_ERR_DEVICE_INDEX there.  Read (and clear) it with
  *     parallax_last_device_error().
- *   - The library keeps one grow-only scratch allocation per device (the fp16
- *     copy of V for the prefill kernel, the split partials for decode).  It
- *     grows with cudaMalloc on first use, so the first call at a new, larger
- *     size must not be inside CUDA graph capture.
+ *   - Scratch.  A call that needs scratch device memory (parallax_fwd on the
+ *     tensor-core path: a work counter and an fp16 copy of V; parallax_decode
+ *     and parallax_decode_paged: the split partials) takes it for that call
+ *     alone from a library-owned, per-device stream-ordered memory pool
+ *     (cudaMallocFromPoolAsync on `stream`) and returns it with cudaFreeAsync
+ *     on `stream` once its kernels are enqueued.  Calls may therefore run
+ *     concurrently on different streams and be made from several host threads
+ *     at once: no two calls share scratch, and nothing is freed while a kernel
+ *     may still use it.  The pool keeps returned memory for later calls.
+ *     parallax_decode_ex (caller's workspace) and parallax_decode_noalloc
+ *     (static array) do not use the pool.
  */
 #ifndef PARALLAX_H
 #define PARALLAX_H
@@ -111,13 +118,16 @@ PARALLAX_API int parallax_fwd(const void *q, const void *k, const void *v, const
  *   y              : [B, H, d] of out_dtype (F32 or BF16).
  *   lse            : [B, H] fp32, may be NULL.
  *   B, H >= 1; Tcap >= 1; d in {64, 128}; in_dtype must be BF16.
- * Uses the library's scratch for split partials; see parallax_decode_ex.
+ * Split partials use per-call scratch from the library's pool (see the
+ * conventions above); calls on different streams may overlap.  See
+ * parallax_decode_ex for caller-provided scratch.
  */
 PARALLAX_API int parallax_decode(const void *q, const void *rho, const void *kcache, const void *vcache,
                     const int *seqlens, void *y, float *lse, int B, int H, int Tcap, int d,
                     int in_dtype, int out_dtype, parallax_stream_t stream);
 
-/* Bytes of scratch parallax_decode_ex needs for this shape (0 if it needs none). */
+/* Bytes of scratch parallax_decode_ex needs for this shape on the current
+ * device (0 if it needs none, or on a bad shape or CUDA error). */
 PARALLAX_API size_t parallax_decode_workspace_bytes(int B, int H, int Tcap, int d);
 
 /*
@@ -154,9 +164,8 @@ PARALLAX_API int parallax_decode_ex(const void *q, const void *rho, const void *
  *   y              : [B, Hq, d] of out_dtype (F32 or BF16); lse [B, Hq] fp32 or NULL.
  *   B, Hkv >= 1; Hq a multiple of Hkv; page_size a power of two in [16, 4096];
  *   max_pages, num_pages >= 1; d in {64, 128}; in_dtype BF16.
- * Split partials use the library's scratch, which grows on demand (a
- * cudaMalloc, after a device synchronization, the first time a shape needs
- * more).  Calls sharing the library's scratch must be ordered on the device.
+ * Split partials use per-call scratch from the library's pool (see the
+ * conventions above); calls on different streams may overlap.
  */
 PARALLAX_API int parallax_decode_paged(const void *q, const void *rho, const void *kpages, const void *vpages,
                                        const int *block_table, const int *seqlens, void *y, float *lse, int B,

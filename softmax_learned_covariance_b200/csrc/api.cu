@@ -1,9 +1,20 @@
 // api.cu -- the C ABI declared in include/parallax.h.
 //
-// Host side only: argument validation, per-device state (device error word,
-// grow-only scratch), TMA descriptor encoding and kernel launches.  Every
-// compute step runs in the CUDA kernels of this directory; there is no host
-// fallback.
+// Host side only: argument validation, per-device state (device error word and
+// a stream-ordered memory pool for per-call scratch), TMA descriptor encoding
+// and kernel launches.  Every compute step runs in the CUDA kernels of this
+// directory; there is no host fallback.
+//
+// Scratch.  A call that needs scratch (the fp16 copy of V and the work counter
+// of the prefill, the split partials of the decodes) takes it from the
+// library's pool with cudaMallocFromPoolAsync on the call's own stream and
+// hands it back with cudaFreeAsync on that stream right after enqueueing its
+// kernels.  Stream order therefore keeps the memory alive exactly as long as
+// the call's kernels run: calls on different streams, or from different host
+// threads, never share scratch, and no buffer is ever freed while a kernel that
+// was handed it may still run.  The pool keeps freed memory for reuse (its
+// release threshold is unlimited), so steady-state calls do not reach the
+// driver's allocator.
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
@@ -24,10 +35,8 @@ constexpr int MAX_DEVICES = 64;
 struct DevState {
     bool init = false;
     int sms = 0;
-    int *err = nullptr;           // device error word (ctl[0])
-    int *counter = nullptr;       // persistent-grid work counter (ctl[32])
-    void *ws = nullptr;
-    size_t ws_bytes = 0;
+    int *err = nullptr;              // device error word
+    cudaMemPool_t pool = nullptr;    // per-call scratch, stream-ordered
 };
 
 std::mutex g_mu;
@@ -45,34 +54,50 @@ int get_state(DevState **out) {
         if (cudaDeviceGetAttribute(&s.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return PARALLAX_ERR_CUDA;
         if (cudaMalloc(&s.err, 256) != cudaSuccess) return PARALLAX_ERR_CUDA;
         if (cudaMemset(s.err, 0, 256) != cudaSuccess) return PARALLAX_ERR_CUDA;
-        s.counter = s.err + 32;
+        cudaMemPoolProps props;
+        std::memset(&props, 0, sizeof(props));
+        props.allocType = cudaMemAllocationTypePinned;
+        props.handleTypes = cudaMemHandleTypeNone;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        if (cudaMemPoolCreate(&s.pool, &props) != cudaSuccess) return PARALLAX_ERR_CUDA;
+        unsigned long long keep = ~0ull;
+        if (cudaMemPoolSetAttribute(s.pool, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess)
+            return PARALLAX_ERR_CUDA;
         s.init = true;
     }
     *out = &s;
     return PARALLAX_OK;
 }
 
-// Grow-only scratch; the old buffer is released after the device is idle.
-int get_workspace(DevState *s, size_t bytes, void **out) {
-    std::lock_guard<std::mutex> lk(g_mu);
-    if (bytes == 0) {
-        *out = s->ws;
+// Scratch of one call: taken from the pool in the call's stream order, given
+// back in the same order when this object goes out of scope (after the call
+// has enqueued its kernels, so the free runs after them on the device).
+class CallScratch {
+  public:
+    CallScratch(const DevState *s, cudaStream_t st) : s_(s), st_(st) {}
+    CallScratch(const CallScratch &) = delete;
+    CallScratch &operator=(const CallScratch &) = delete;
+    ~CallScratch() {
+        if (p_) cudaFreeAsync(p_, st_);
+    }
+    // 256-byte aligned device memory of at least `bytes` (nullptr for 0 bytes).
+    int get(size_t bytes, void **out) {
+        *out = nullptr;
+        if (bytes == 0) return PARALLAX_OK;
+        if (cudaMallocFromPoolAsync(&p_, bytes, s_->pool, st_) != cudaSuccess) {
+            p_ = nullptr;
+            return PARALLAX_ERR_CUDA;
+        }
+        *out = p_;
         return PARALLAX_OK;
     }
-    if (s->ws_bytes < bytes) {
-        if (s->ws) {
-            if (cudaDeviceSynchronize() != cudaSuccess) return PARALLAX_ERR_CUDA;
-            cudaFree(s->ws);
-            s->ws = nullptr;
-            s->ws_bytes = 0;
-        }
-        const size_t want = (bytes + (1u << 20) - 1) & ~(size_t)((1u << 20) - 1);
-        if (cudaMalloc(&s->ws, want) != cudaSuccess) return PARALLAX_ERR_CUDA;
-        s->ws_bytes = want;
-    }
-    *out = s->ws;
-    return PARALLAX_OK;
-}
+
+  private:
+    const DevState *s_;
+    cudaStream_t st_;
+    void *p_ = nullptr;
+};
 
 }  // namespace
 
@@ -191,8 +216,12 @@ int parallax_fwd(const void *q, const void *k, const void *v, const void *rho, v
 
     if ((st = ensure_encoder())) return st;
     const size_t n = (size_t)B * H * T * d;
-    void *v16 = nullptr;
-    if ((st = get_workspace(s, n * 2, &v16))) return st;
+    // scratch: the persistent grid's work counter, then the fp16 copy of V
+    CallScratch scratch(s, cs);
+    void *ws = nullptr;
+    if ((st = scratch.get(256 + n * 2, &ws))) return st;
+    int *counter = static_cast<int *>(ws);
+    void *v16 = static_cast<char *>(ws) + 256;
     if (launch_convert_bf16_to_f16(v, v16, n, cs) != cudaSuccess) return PARALLAX_ERR_CUDA;
 
     FwdTensorMaps tm;
@@ -208,7 +237,7 @@ int parallax_fwd(const void *q, const void *k, const void *v, const void *rho, v
         tm.r = tm.q;
     }
     return status_of(
-        launch_fwd_sm100(tm, rho != nullptr, y, lse, B, H, T, d, causal, out_dtype, s->sms, s->counter, make_ctl(s), cs));
+        launch_fwd_sm100(tm, rho != nullptr, y, lse, B, H, T, d, causal, out_dtype, s->sms, counter, make_ctl(s), cs));
 }
 
 size_t parallax_decode_workspace_bytes(int B, int H, int Tcap, int d) {
@@ -235,8 +264,9 @@ static int decode_impl(const void *q, const void *rho, const void *kcache, const
     const DecodePlan plan = plan_decode(B, H, Tcap, d, s->sms);
     const size_t need = decode_partials_bytes(B, H, d, plan);
     void *ws = nullptr;
+    CallScratch scratch(s, static_cast<cudaStream_t>(stream));
     if (own_workspace) {
-        if ((st = get_workspace(s, need, &ws))) return st;
+        if ((st = scratch.get(need, &ws))) return st;
     } else {
         if (need > 0 && (!workspace)) return PARALLAX_ERR_NULL;
         if (workspace_bytes < need) return PARALLAX_ERR_SHAPE;
@@ -277,7 +307,8 @@ int parallax_decode_paged(const void *q, const void *rho, const void *kpages, co
     const int Tcap = max_pages * page_size;
     const DecodePlan plan = plan_decode_paged(B, Hq, Hkv, Tcap, d, s->sms);
     void *ws = nullptr;
-    if ((st = get_workspace(s, decode_partials_bytes(B, Hq, d, plan), &ws))) return st;
+    CallScratch scratch(s, static_cast<cudaStream_t>(stream));
+    if ((st = scratch.get(decode_partials_bytes(B, Hq, d, plan), &ws))) return st;
     const PagedKV pg{block_table, max_pages, num_pages, pshift, Hkv, Hq / Hkv};
     return status_of(launch_decode_paged(q, rho, kpages, vpages, pg, seqlens, y, lse, B, Hq, d, out_dtype, plan,
                                          static_cast<float *>(ws), make_ctl(s), static_cast<cudaStream_t>(stream)));

@@ -395,29 +395,6 @@ cudaError_t launch_t(const void *q, const void *rho, const void *kc, const void 
 
 }  // namespace
 
-DecodePlan plan_decode(int B, int H, int Tcap, int d, int sm_count) {
-    (void)d;
-    DecodePlan p;
-    const long bh = (long)B * H;
-    // About 64 units per SM (4 waves of resident CTAs) so the block scheduler
-    // can balance ragged lengths; chunks are multiples of 128 tokens (a unit's
-    // partial state is 2d + 3 floats, ~1% of a 128-token chunk's K/V bytes).
-    const long want_units = 64L * sm_count;
-    long nsplit = want_units / bh;
-    if (nsplit < 1) nsplit = 1;
-    long chunk = ((long)Tcap + nsplit - 1) / nsplit;
-    chunk = ((chunk + 127) / 128) * 128;
-    if (chunk >= Tcap) chunk = Tcap;                 // one unit per sequence
-    p.chunk = (int)chunk;
-    p.nsplit = (int)(((long)Tcap + chunk - 1) / chunk);
-    return p;
-}
-
-size_t decode_partials_bytes(int B, int H, int d, const DecodePlan &p) {
-    if (p.nsplit <= 1) return 0;
-    return (size_t)B * H * p.nsplit * (2 * d + 3) * sizeof(float);
-}
-
 cudaError_t launch_decode(const void *q, const void *rho, const void *kc, const void *vc, const int *seqlens,
                           void *y, float *lse, int B, int H, int Tcap, int d, int out_dtype, const DecodePlan &p,
                           float *partials, int sm_count, const DeviceCtl &ctl, cudaStream_t s) {
@@ -431,14 +408,6 @@ cudaError_t launch_decode(const void *q, const void *rho, const void *kc, const 
     if (out_dtype == PARALLAX_F32)
         return launch_t<128, float>(q, rho, kc, vc, seqlens, y, lse, B, H, Tcap, p, partials, s);
     return launch_t<128, __nv_bfloat16>(q, rho, kc, vc, seqlens, y, lse, B, H, Tcap, p, partials, s);
-}
-
-DecodePlan plan_decode_paged(int B, int Hq, int Hkv, int Tcap, int d, int sm_count) {
-    // a 4-warp tensor-core unit serves up to 8 query heads of a KV head; it is
-    // sized like four split-kernel units so that each warp streams enough
-    // tiles to amortise its pipeline fill and the final merge
-    const int group = Hq / Hkv;
-    return plan_decode(B, Hkv * ((group + 7) / 8) * 4, Tcap, d, sm_count);
 }
 
 cudaError_t launch_decode_paged(const void *q, const void *rho, const void *kpages, const void *vpages,

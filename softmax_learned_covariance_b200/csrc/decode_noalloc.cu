@@ -5,9 +5,11 @@
 // start-up and run under a fixed budget, latency-critical decode loops where a
 // cudaMalloc or the device-wide synchronization of a cudaFree would stall every
 // stream, and plugin interfaces whose execute callbacks forbid allocation.
-// parallax_decode grows a library scratch buffer with cudaMalloc on first use;
-// this entry point instead keeps the split partials in a fixed-size array
-// compiled into the library, so it never allocates.
+// parallax_decode takes its scratch from a library memory pool with a
+// stream-ordered allocation per call, which reaches the driver's allocator
+// whenever the pool has to grow; this entry point instead keeps the split
+// partials in a fixed-size array compiled into the library, so it never
+// allocates.
 //
 // The array lives in device memory of every GPU that loads the library and
 // stays there until the process exits.  In host code its name is only a
@@ -25,6 +27,12 @@ namespace {
 
 constexpr size_t kScratchBytes = PARALLAX_DECODE_NOALLOC_SCRATCH_BYTES;
 constexpr int kMaxDevices = 64;
+// The split plan caps the partials at 64 units per SM of 2d + 3 floats, so on
+// any device with up to this many SMs (a B200 has 148) every shape fits and the
+// size check below never rejects.
+constexpr int kSmsAlwaysFit = 252;
+static_assert(plx::decode_partials_bound(kSmsAlwaysFit, 128) <= kScratchBytes,
+              "the static decode scratch must hold the partials of every shape on these devices");
 
 // Shared by every call on a device; keeps the last call's contents.
 static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];

@@ -80,6 +80,7 @@ constexpr float LN2 = 0.6931471805599453f;
 constexpr float RESCALE_THRESHOLD = 8.0f;   // log2 units
 constexpr float A_SCALE = 1.0f / 256.0f;
 constexpr float A_UNSCALE = 256.0f;
+constexpr unsigned long long DRAIN_NS = 2000000ull;   // bound of the exit-time drain waits
 
 constexpr int Q_BYTES = BM * D * 2;       // 32 KB: two 64-column halves of [128 rows x 128 B]
 constexpr int K_BYTES = BN * D * 2;       // 32 KB: two halves of [128 keys x 128 B]
@@ -111,6 +112,7 @@ struct __align__(8) Bars {
     uint64_t om_free;             // epilogue has read O and M
     uint64_t xchg[2];             // per tile parity: every softmax warp posted its partial max
     uint64_t esum;                // per item: partial sums posted
+    uint64_t drain[2];            // last commit of each UMMA issuer (all its MMAs complete)
     uint64_t sched_full[SCHED], sched_empty[SCHED];
     int sched_item[SCHED];
     uint32_t tmem_base;
@@ -239,6 +241,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_init(smem_u32(&bars->xchg[0]), NSOFT_WARPS);
         mbar_init(smem_u32(&bars->xchg[1]), NSOFT_WARPS);
         mbar_init(smem_u32(&bars->esum), NSOFT_WARPS);
+        mbar_init(smem_u32(&bars->drain[0]), 1);
+        mbar_init(smem_u32(&bars->drain[1]), 1);
         for (int s = 0; s < SCHED; ++s) {
             mbar_init(smem_u32(&bars->sched_full[s]), 1);
             mbar_init(smem_u32(&bars->sched_empty[s]), 3 + NSOFT_WARPS);   // two UMMA threads, V producer, softmax warps
@@ -254,7 +258,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
-    WaitCtl wc{ctl.err, &bars->abort_flag, globaltimer_ns() + ctl.wait_ns};
+    WaitCtl wc{ctl.err, &bars->abort_flag, ctl.wait_ns};
 
     const int nq = (T + BM - 1) / BM;
     const int items = nq * BH;
@@ -265,6 +269,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tma_prefetch_desc(&tm_k);
         if (WITH_RHO) tma_prefetch_desc(&tm_r);
         uint32_t kc = 0;
+        int k_armed[KST], qr_armed = -1;   // parity of each buffer's last fill still to land, -1 if none
+        for (int s = 0; s < KST; ++s) k_armed[s] = -1;
         bool ok = true;
         for (uint32_t ic = 0; ok; ++ic) {
             const uint32_t ss = ic % SCHED;
@@ -277,6 +283,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int q0 = it.qt * BM;
             if (!mbar_wait(smem_u32(&bars->qr_empty), (ic & 1) ^ 1, wc)) break;
             const uint32_t qf = smem_u32(&bars->qr_full);
+            qr_armed = (int)(ic & 1);
             mbar_arrive_expect_tx(qf, WITH_RHO ? 2 * Q_BYTES : Q_BYTES);
             tma_load_3d(sbase + OFF_Q, &tm_q, qf, 0, q0, it.bh);
             tma_load_3d(sbase + OFF_Q + Q_BYTES / 2, &tm_q, qf, 64, q0, it.bh);
@@ -291,16 +298,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const uint32_t dst = sbase + OFF_K + s * K_BYTES;
                 const bool skip = (ctl.debug_flags & DEBUG_FWD_SKIP_FIRST_K_LOAD) && kc == 0;
                 if (!skip) {
+                    k_armed[s] = (int)((kc / KST) & 1);
                     mbar_arrive_expect_tx(f, K_BYTES);
                     tma_load_3d(dst, &tm_k, f, 0, j * BN, it.bh);
                     tma_load_3d(dst + K_BYTES / 2, &tm_k, f, 64, j * BN, it.bh);
                 }
             }
         }
+        // no copy of this thread may still be landing when the CTA exits
+        if (qr_armed >= 0) mbar_wait_drain(smem_u32(&bars->qr_full), (uint32_t)qr_armed, DRAIN_NS);
+        for (int s = 0; s < KST; ++s)
+            if (k_armed[s] >= 0) mbar_wait_drain(smem_u32(&bars->k_full[s]), (uint32_t)k_armed[s], DRAIN_NS);
     } else if (warp == V_WARP && lane == 0) {
         // ==================================================== V producer ==
         tma_prefetch_desc(&tm_v);
         uint32_t vc = 0;
+        int v_armed[VST];
+        for (int s = 0; s < VST; ++s) v_armed[s] = -1;
         bool ok = true;
         for (uint32_t ic = 0; ok; ++ic) {
             int w;
@@ -313,6 +327,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     const int s = vc % VST;
                     if (!mbar_wait(smem_u32(&bars->v_empty[s]), ((vc / VST) & 1) ^ 1, wc)) { ok = false; break; }
                     const uint32_t f = smem_u32(&bars->v_full[s]);
+                    v_armed[s] = (int)((vc / VST) & 1);
                     const uint32_t dst = sbase + OFF_V + s * V_BYTES;
                     mbar_arrive_expect_tx(f, V_BYTES);
                     tma_load_3d(dst, &tm_v, f, 0, j * BN + vs * VKEYS, it.bh);
@@ -320,6 +335,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
             }
         }
+        for (int s = 0; s < VST; ++s)
+            if (v_armed[s] >= 0) mbar_wait_drain(smem_u32(&bars->v_full[s]), (uint32_t)v_armed[s], DRAIN_NS);
     } else if (warp == 1 && lane == 0) {
         // ============================================= score UMMA issuer ==
         // Per key tile j: S(j) into X once the softmax has loaded A(j-1)
@@ -368,6 +385,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (j == it.nkv - 1) tc_commit(smem_u32(&bars->qr_empty));
             }
         }
+        // every MMA this thread issued has completed before TMEM is released
+        tc_commit(smem_u32(&bars->drain[0]));
+        mbar_wait_drain(smem_u32(&bars->drain[0]), 0, DRAIN_NS);
     } else if (warp == PV_WARP && lane == 0) {
         // ============================================== P.V UMMA issuer ==
         uint32_t vc = 0, G = 0;
@@ -406,6 +426,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (ok) tc_commit(smem_u32(&bars->pv_done));
             }
         }
+        tc_commit(smem_u32(&bars->drain[1]));
+        mbar_wait_drain(smem_u32(&bars->drain[1]), 0, DRAIN_NS);
     } else if (warp >= FIRST_SOFT_WARP && warp < PV_WARP) {
         // ============================================ softmax + epilogue ==
         const int grp = (warp - FIRST_SOFT_WARP) >> 2;   // key columns [32 grp, 32 grp + 32)
@@ -609,7 +631,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
 
     __syncthreads();
-    if (bars->abort_flag) __nanosleep(100000);   // let in-flight copies and MMAs land
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);

@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "decode_plan.h"
 #include "parallax.h"
 
 namespace plx {
@@ -40,13 +41,7 @@ cudaError_t launch_convert_bf16_to_f16(const void *src, void *dst, size_t n, cud
 cudaError_t launch_fwd_simt(const void *q, const void *k, const void *v, const void *rho, void *y, float *lse,
                             int B, int H, int T, int d, int causal, int in_dtype, int out_dtype, cudaStream_t s);
 
-// split-KV decode + combine
-struct DecodePlan {
-    int nsplit;      // chunks per sequence (units per head)
-    int chunk;       // tokens per chunk: a multiple of 128, or the whole cache
-};
-DecodePlan plan_decode(int B, int H, int Tcap, int d, int sm_count);
-size_t decode_partials_bytes(int B, int H, int d, const DecodePlan &p);
+// split-KV decode + combine (the split plan is in decode_plan.h)
 cudaError_t launch_decode(const void *q, const void *rho, const void *kc, const void *vc, const int *seqlens,
                           void *y, float *lse, int B, int H, int Tcap, int d, int out_dtype, const DecodePlan &p,
                           float *partials, int sm_count, const DeviceCtl &ctl, cudaStream_t s);
@@ -57,8 +52,6 @@ struct PagedKV {
     const int *table;   // [B, max_pages] page ids (device)
     int max_pages, num_pages, pshift, Hkv, group;
 };
-// Split plan of the paged decode for the kernel that serves this head grouping.
-DecodePlan plan_decode_paged(int B, int Hq, int Hkv, int Tcap, int d, int sm_count);
 // Tensor-core split kernel of the paged decode (any Hq / Hkv); writes the same
 // partials (or y when nsplit == 1) as the split decode kernel.
 cudaError_t launch_decode_gqa_split(const void *q, const void *rho, const void *kpages, const void *vpages,

@@ -34,9 +34,11 @@ struct __align__(8) Bars {
     uint64_t empty[STAGES];
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
+    uint64_t drain;               // the UMMA issuer's last commit (all its MMAs complete)
     uint32_t tmem_base;
     int abort_flag;
 };
+constexpr unsigned long long DRAIN_NS = 2000000ull;   // bound of the exit-time drain waits
 
 constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + (size_t)STAGES * STAGE_BYTES + sizeof(Bars);
 
@@ -57,6 +59,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mbar_init(smem_u32(&bars->acc_full[b]), 1);
             mbar_init(smem_u32(&bars->acc_empty[b]), 128);
         }
+        mbar_init(smem_u32(&bars->drain), 1);
         bars->abort_flag = 0;
         fence_mbar_init();
     }
@@ -69,7 +72,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
 
-    WaitCtl wc{ctl.err, &bars->abort_flag, globaltimer_ns() + ctl.wait_ns};
+    WaitCtl wc{ctl.err, &bars->abort_flag, ctl.wait_ns};
     const int m_tiles = (M + BM - 1) / BM;
     const int n_tiles = N / BN;
     const int tiles = m_tiles * n_tiles;
@@ -80,6 +83,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tma_prefetch_desc(&tm_x);
         tma_prefetch_desc(&tm_w);
         uint32_t it = 0;
+        int armed[STAGES];   // parity of each stage's last fill still to land, -1 if none
+        for (int s = 0; s < STAGES; ++s) armed[s] = -1;
         bool ok = true;
         for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
             const int m0 = (t / n_tiles) * BM, n0 = (t % n_tiles) * BN;
@@ -88,6 +93,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const uint32_t ph = (it / STAGES) & 1;
                 if (!mbar_wait(smem_u32(&bars->empty[s]), ph ^ 1, wc)) { ok = false; break; }
                 const uint32_t full = smem_u32(&bars->full[s]);
+                armed[s] = (int)ph;
                 mbar_arrive_expect_tx(full, STAGE_BYTES);
                 const uint32_t sa = smem_u32(smem + (size_t)s * STAGE_BYTES);
                 const uint32_t sb = sa + A_BYTES;
@@ -96,6 +102,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 for (int g = 0; g < BN / 64; ++g) tma_load_2d(sb + g * (BK * 128), &tm_w, full, n0 + g * 64, kb * BK);
             }
         }
+        // no copy of this thread may still be landing when the CTA exits
+        for (int s = 0; s < STAGES; ++s)
+            if (armed[s] >= 0) mbar_wait_drain(smem_u32(&bars->full[s]), (uint32_t)armed[s], DRAIN_NS);
     } else if (warp == 1 && lane == 0) {
         // ------------------------------------------------- UMMA issuer --
         uint32_t it = 0, local = 0;
@@ -122,6 +131,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             if (ok) tc_commit(smem_u32(&bars->acc_full[ab]));
         }
+        // every MMA this thread issued has completed before TMEM is released
+        tc_commit(smem_u32(&bars->drain));
+        mbar_wait_drain(smem_u32(&bars->drain), 0, DRAIN_NS);
     } else if (warp >= 4) {
         // ---------------------------------------------------- epilogue --
         const int quarter = warp & 3;
@@ -164,7 +176,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
 
     __syncthreads();
-    if (bars->abort_flag) __nanosleep(100000);   // let in-flight copies and MMAs land
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);

@@ -1,9 +1,12 @@
 // sm100.cuh -- thin inline-PTX wrappers for sm_100a: mbarrier, TMA, tcgen05.
 //
 // Every wait here is bounded: it polls with try_wait and checks %globaltimer;
-// past the deadline it records PARALLAX_ERR_DEVICE_TIMEOUT in the device error
-// word, raises the CTA's abort flag and returns false.  A waiter also returns
-// false early when another thread of the CTA has raised the abort flag.
+// when one wait has lasted longer than the budget it records
+// PARALLAX_ERR_DEVICE_TIMEOUT in the device error word, raises the CTA's abort
+// flag and returns false.  The budget applies to each wait on its own (counted
+// from the wait's first unsuccessful poll), so a long but healthy kernel never
+// runs out of it.  A waiter also returns false early when another thread of the
+// CTA has raised the abort flag.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -15,7 +18,7 @@ namespace plx {
 struct WaitCtl {
     int *err;                      // device error word (global)
     volatile int *abort_flag;      // CTA abort flag (shared)
-    unsigned long long deadline;   // %globaltimer value after which waits give up
+    unsigned long long wait_ns;    // budget of one wait, nanoseconds
 };
 
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
@@ -61,15 +64,31 @@ static __device__ __noinline__ void record_timeout(const WaitCtl &w) {
 // Wait for the phase with the given parity to complete.  False on timeout/abort.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtl &w) {
     if (mbar_try_wait(bar, parity)) return true;
+    unsigned long long t0 = 0;
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 255u) == 0) {
             if (*w.abort_flag) return false;
-            if (globaltimer_ns() > w.deadline) {
+            const unsigned long long now = globaltimer_ns();
+            if (t0 == 0) {
+                t0 = now;
+            } else if (now - t0 > w.wait_ns) {
                 record_timeout(w);
                 return false;
             }
         }
+    }
+}
+
+// Wait used while draining after an abort: ignores the abort flag (the point
+// is to let copies and MMAs already in flight land) and gives up silently
+// after `ns`.  True if the phase completed.
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, unsigned long long ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 63u) == 0 && globaltimer_ns() - t0 > ns) return false;
     }
 }
 

@@ -111,6 +111,45 @@ def fwd_bf16_inputs(B, H, T, d, rho_scale=0.905, seed=3):
     return q, k, v, rho
 
 
+def fwd_rescale_inputs(B, H, T, d, rho_scale=0.905, groups=8, spike=6.0, seed=11):
+    """bf16 forward inputs whose running row max rises after the first key tile.
+
+    Query row i belongs to group g = i % groups and is q_i = sqrt(d) e_g + 0.3 n
+    (e_g the g-th unit vector, n ~ N(0,1)^d).  Keys are small, k ~ N(0, 0.05^2),
+    so background scores are ~0 and every visible key keeps a weight near 1.
+    For each group, one planted key k = spike * e_g in key tile 1 + 4g mod (tiles - 1)
+    (128-key tiles) gives that group's rows a score of ~spike (6 nats = 8.7 in
+    log2 units); for odd groups a second planted key one tile later scores
+    ~2 * spike.  Rows of other groups score those keys at ~0.  v ~ N(0,1);
+    rho ~ N(0, rho_scale^2).  Returns (q, k, v, rho, spikes) where spikes lists
+    (group, key index, score) for each planted key.
+    """
+    rng = np.random.default_rng(seed)
+    shape = (B, H, T, d)
+    grp = np.arange(T) % groups
+    q = rng.standard_normal(size=shape) * 0.3
+    q[..., np.arange(T), grp] += np.sqrt(d)
+    k = rng.standard_normal(size=shape) * 0.05
+    v = rng.standard_normal(size=shape)
+    rho = rng.standard_normal(size=shape) * rho_scale
+    spikes = []
+    ntiles = (T + 127) // 128
+    if ntiles >= 2:
+        for g in range(groups):
+            t1 = 1 + (4 * g) % (ntiles - 1)
+            j1 = min(T - 1, t1 * 128 + (17 * g) % 128)
+            k[..., j1, :] = 0.0
+            k[..., j1, g] = spike
+            spikes.append((g, j1, spike))
+            if g % 2 == 1 and t1 + 1 < ntiles:
+                j2 = min(T - 1, (t1 + 1) * 128 + (29 * g) % 128)
+                k[..., j2, :] = 0.0
+                k[..., j2, g] = 2 * spike
+                spikes.append((g, j2, 2 * spike))
+    return (Tensor16(bf16_bits(q)), Tensor16(bf16_bits(k)), Tensor16(bf16_bits(v)), Tensor16(bf16_bits(rho)),
+            spikes)
+
+
 def rho_proj_inputs(B, T, d_model=2048, H=16, d=128, w_scale=0.02, seed=3):
     """x ~ N(0,1) [B,T,d_model] and W_R ~ N(0, w_scale^2) [d_model, H*d], both bf16."""
     rng = np.random.default_rng(seed + 1000)

@@ -83,3 +83,28 @@ def test_sweep_cell_sampled_heads():
     yr, lr = oracle.decode(q.f64, rho.f64, kc.f64, vc.f64, sl, bh_list=bh)
     parity.assert_bf16_parity(y.cpu().numpy().reshape(B * H, d)[bh], yr, 1, "sweep cell")
     parity.assert_lse(lse.cpu().numpy().reshape(-1)[bh], lr)
+
+
+@pytest.mark.parametrize("B,ctx", [(1, 32768), (8, 8192)])
+def test_long_context_cells_sampled_heads(B, ctx):
+    """Long-context cells of the decode sweep with ragged lengths in [ctx/2, ctx]:
+    B=1 ctx 32768 (one head is split into up to 256 chunks, merged by the
+    16-warp combine) and B=8 ctx 8192.  Inputs drawn on the device with a
+    seeded generator; sampled heads read back and checked against the oracle."""
+    H, d = 16, 128
+    sl = inputs.ragged_seqlens(B, ctx, 4 + 100 + B)
+    q, r, kc, vc, ds = inputs.decode_inputs_device(B, H, ctx, d, sl, seed=4 + 100 + B, device=DEV)
+    y, lse = plx.parallax_decode(q, r, kc, vc, ds)
+    torch.cuda.synchronize()
+    assert plx.parallax_last_device_error() == 0
+    heads = [(b, h) for b in range(B) for h in (0, 7, 15)]
+
+    def host(t):
+        return inputs.Tensor16(t.contiguous().cpu().view(torch.int16).numpy().view(np.uint16))
+
+    for b, h in heads:
+        hq, hr = host(q[b:b + 1, h:h + 1]), host(r[b:b + 1, h:h + 1])
+        hk, hv = host(kc[b:b + 1, h:h + 1]), host(vc[b:b + 1, h:h + 1])
+        yr, lr = oracle.decode(hq.f64, hr.f64, hk.f64, hv.f64, sl[b:b + 1])
+        parity.assert_bf16_parity(y[b:b + 1, h:h + 1].cpu().numpy(), yr, 2, f"B={B} ctx={ctx} head {b},{h}")
+        parity.assert_lse(lse[b:b + 1, h:h + 1].cpu().numpy(), lr)

@@ -107,3 +107,24 @@ def test_long_prefill_t32768_and_softmax_identity():
     y0, l0 = _run_bf16(q, k, v, zero)
     yn, ln = _run_bf16(q, k, v, None)
     assert torch.equal(y0, yn) and torch.equal(l0, ln)
+
+
+@pytest.mark.parametrize("T", [300, 4096])
+@pytest.mark.parametrize("causal", [True, False])
+def test_bf16_row_max_rises_after_the_first_tile(T, causal):
+    """Planted keys lift rows' running max by > 8 log2 units in later key tiles
+    (once or twice), so the kernel rescales O and M in TMEM while earlier tiles
+    still carry much of the weight; y and lse against the oracle, and rho = 0
+    bitwise equal to the softmax-only instantiation on the same inputs."""
+    q, k, v, rho, spikes = inputs.fwd_rescale_inputs(1, 2, T, 128, seed=11 + T)
+    assert spikes
+    y, lse = _run_bf16(q, k, v, rho, causal)
+    yr, lr = oracle.fwd(q.f64, k.f64, v.f64, rho.f64, causal=causal)
+    parity.assert_bf16_parity(y.cpu().numpy(), yr, 2, f"rescale T={T} causal={causal}")
+    parity.assert_lse(lse.cpu().numpy(), lr, f"rescale T={T} lse")
+    zero = inputs.Tensor16(np.zeros_like(q.bits))
+    y0, l0 = _run_bf16(q, k, v, zero, causal)
+    yn, ln = _run_bf16(q, k, v, None, causal)
+    assert torch.equal(y0, yn) and torch.equal(l0, ln)
+    ys, _ = oracle.fwd(q.f64, k.f64, v.f64, None, causal=causal)
+    parity.assert_bf16_parity(yn.cpu().numpy(), ys, 2, f"rescale softmax-only T={T}")

@@ -49,3 +49,25 @@ def test_paged_decode_inputs_shapes_and_table():
     # deterministic in the seed
     again = inputs.paged_decode_inputs(3, 8, 2, 32, 5, 64, sl, seed=1, spare_pages=4)
     assert np.array_equal(again[4], table) and np.array_equal(again[2].bits, kp.bits)
+
+
+def test_rescale_inputs_raise_the_row_max_after_the_first_tile():
+    """The planted keys lift a row's max score by > 8 in log2 units in a later
+    128-key tile (one or two rises), while the keys before the rise still hold
+    a sizeable share of the softmax weight, for causal and full rows alike."""
+    T, d = 4096, 128
+    q, k, v, rho, spikes = inputs.fwd_rescale_inputs(1, 1, T, d, seed=11)
+    z = (q.f64[0, 0] @ k.f64[0, 0].T) / np.sqrt(d) * np.log2(np.e)
+    assert len(spikes) >= 8
+    for causal in (True, False):
+        zc = np.where(np.tril(np.ones((T, T), bool)), z, -np.inf) if causal else z
+        tmax = np.maximum.accumulate(zc.reshape(T, T // 128, 128).max(axis=2), axis=1)
+        rises = (np.diff(tmax, axis=1) > 8).sum(axis=1)
+        assert np.mean(rises >= 1) > 0.4 and np.any(rises >= 2)
+        # weight share of the keys before a row's first rise: the part of O and
+        # M that the rescale multiplies; it must be large for many rows
+        w = np.exp2(zc - zc.max(axis=1, keepdims=True))
+        first = np.argmax(np.diff(tmax, axis=1) > 8, axis=1) + 1
+        rows = np.nonzero(rises >= 1)[0]
+        before = np.array([w[i, :first[i] * 128].sum() / w[i].sum() for i in rows[::7]])
+        assert np.quantile(before, 0.9) > 0.2 and before.max() > 0.3
