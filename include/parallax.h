@@ -28,12 +28,14 @@
  *   - Device-side waits are bounded.  A wait that gives up records
  *     PARALLAX_ERR_DEVICE_TIMEOUT in a per-device error word and the kernel
  *     returns; an out-of-range page id met by the paged decode records
- *     PARALLAX_ERR_DEVICE_INDEX there.  Read (and clear) it with
+ *     PARALLAX_ERR_DEVICE_INDEX there, and a non-finite prefill output
+ *     PARALLAX_ERR_DEVICE_RANGE.  Read (and clear) it with
  *     parallax_last_device_error().
  *   - Scratch.  A call that needs scratch device memory (parallax_fwd on the
- *     tensor-core path: a work counter and an fp16 copy of V; parallax_decode
- *     and parallax_decode_paged: the split partials) takes it for that call
- *     alone from a library-owned, per-device stream-ordered memory pool
+ *     tensor-core path: a work counter and a block-scaled fp16 copy of V;
+ *     parallax_decode and parallax_decode_paged: the split partials) takes it
+ *     for that call alone from a library-owned, per-device stream-ordered
+ *     memory pool
  *     (cudaMallocFromPoolAsync on `stream`) and returns it with cudaFreeAsync
  *     on `stream` once its kernels are enqueued.  Calls may therefore run
  *     concurrently on different streams and be made from several host threads
@@ -73,7 +75,8 @@ typedef enum {
     PARALLAX_ERR_UNSUPPORTED = 5,    /* valid request this build does not serve */
     PARALLAX_ERR_CUDA = 6,           /* a CUDA runtime/driver call failed */
     PARALLAX_ERR_DEVICE_TIMEOUT = 7, /* a device-side wait gave up */
-    PARALLAX_ERR_DEVICE_INDEX = 8    /* a device-side index (a page id) was out of range */
+    PARALLAX_ERR_DEVICE_INDEX = 8,   /* a device-side index (a page id) was out of range */
+    PARALLAX_ERR_DEVICE_RANGE = 9    /* a result was not finite: an input outside the kernel's range */
 } parallax_status_t;
 
 /*
@@ -96,8 +99,15 @@ typedef enum {
  *     F32  -> F32   fp32 CUDA-core kernel (fp32 arithmetic throughout)
  *     BF16 -> F32   tensor-core kernel (tcgen05), fp32 accumulation
  *     BF16 -> BF16  same kernel, y rounded to bf16 on store
- *   Tensor-core path constraints: d == 128, |k_j . rho_i| < 65504 (the
- *   correction weights are staged in fp16), |v| < 65504.
+ *   Tensor-core path: d in {64, 128}.  The P.V products run on fp16 operands:
+ *   V is converted to fp16 with a power-of-two scale per block of 64 keys,
+ *   which keeps fp16 precision for |v| from about 1e-5 (smaller values lose
+ *   precision gradually) up to |v| < 2^23; the correction weights
+ *   P o (k_j . rho_i) / 256 are staged in fp16, so |k_j . rho_i| < 65504
+ *   (divided by 2^e in a block where V needed a scale 2^-e, e <= 7).  A
+ *   non-finite output (an input outside these ranges, or a non-finite input)
+ *   sets PARALLAX_ERR_DEVICE_RANGE in the device error word.  Scratch: 2 bytes
+ *   per V element plus a few bytes (see the conventions above).
  */
 PARALLAX_API int parallax_fwd(const void *q, const void *k, const void *v, const void *rho,
                  void *y, float *lse, int B, int H, int T, int d, int causal,

@@ -5,8 +5,9 @@
 // and kernel launches.  Every compute step runs in the CUDA kernels of this
 // directory; there is no host fallback.
 //
-// Scratch.  A call that needs scratch (the fp16 copy of V and the work counter
-// of the prefill, the split partials of the decodes) takes it from the
+// Scratch.  A call that needs scratch (the prefill's work counter and
+// block-scaled fp16 copy of V, the split partials of the decodes) takes it
+// from the
 // library's pool with cudaMallocFromPoolAsync on the call's own stream and
 // hands it back with cudaFreeAsync on that stream right after enqueueing its
 // kernels.  Stream order therefore keeps the memory alive exactly as long as
@@ -167,6 +168,7 @@ const char *parallax_strerror(int status) {
         case PARALLAX_ERR_CUDA: return "a CUDA call failed";
         case PARALLAX_ERR_DEVICE_TIMEOUT: return "a device-side wait gave up (bounded wait expired)";
         case PARALLAX_ERR_DEVICE_INDEX: return "a device-side index (a page id) was out of range";
+        case PARALLAX_ERR_DEVICE_RANGE: return "a result was not finite (an input outside the kernel's range)";
         default: return "unknown status";
     }
 }
@@ -205,7 +207,6 @@ int parallax_fwd(const void *q, const void *k, const void *v, const void *rho, v
     const bool f32 = in_dtype == PARALLAX_F32 && out_dtype == PARALLAX_F32;
     const bool bf16 = in_dtype == PARALLAX_BF16 && (out_dtype == PARALLAX_F32 || out_dtype == PARALLAX_BF16);
     if (!f32 && !bf16) return PARALLAX_ERR_DTYPE;
-    if (bf16 && d != 128) return PARALLAX_ERR_UNSUPPORTED;
 
     DevState *s = nullptr;
     int st = get_state(&s);
@@ -215,14 +216,17 @@ int parallax_fwd(const void *q, const void *k, const void *v, const void *rho, v
     if (f32) return status_of(launch_fwd_simt(q, k, v, rho, y, lse, B, H, T, d, causal, in_dtype, out_dtype, cs));
 
     if ((st = ensure_encoder())) return st;
+    // scratch: the persistent grid's work counter, the block exponents of V,
+    // and V as block-scaled fp16
     const size_t n = (size_t)B * H * T * d;
-    // scratch: the persistent grid's work counter, then the fp16 copy of V
+    const size_t nexp = ((size_t)B * H * v16_blocks(T) + 255) & ~(size_t)255;
     CallScratch scratch(s, cs);
     void *ws = nullptr;
-    if ((st = scratch.get(256 + n * 2, &ws))) return st;
+    if ((st = scratch.get(256 + nexp + n * 2, &ws))) return st;
     int *counter = static_cast<int *>(ws);
-    void *v16 = static_cast<char *>(ws) + 256;
-    if (launch_convert_bf16_to_f16(v, v16, n, cs) != cudaSuccess) return PARALLAX_ERR_CUDA;
+    signed char *vexp = static_cast<signed char *>(ws) + 256;
+    void *v16 = static_cast<char *>(ws) + 256 + nexp;
+    if (launch_v_to_f16_blocks(v, v16, vexp, B * H, T, d, cs) != cudaSuccess) return PARALLAX_ERR_CUDA;
 
     FwdTensorMaps tm;
     const uint64_t dims[3] = {(uint64_t)d, (uint64_t)T, (uint64_t)B * H};
@@ -230,14 +234,16 @@ int parallax_fwd(const void *q, const void *k, const void *v, const void *rho, v
     const uint32_t box_q[3] = {64, 128, 1}, box_k[3] = {64, 128, 1}, box_v[3] = {64, 64, 1};
     if ((st = encode(&tm.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, 3, dims, box_q, 2))) return st;
     if ((st = encode(&tm.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k, 3, dims, box_k, 2))) return st;
-    if ((st = encode(&tm.v16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, v16, 3, dims, box_v, 2))) return st;
+    if ((st = encode(&tm.v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, v16, 3, dims, box_v, 2))) return st;
+
     if (rho) {
         if ((st = encode(&tm.r, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rho, 3, dims, box_q, 2))) return st;
     } else {
         tm.r = tm.q;
     }
     return status_of(
-        launch_fwd_sm100(tm, rho != nullptr, y, lse, B, H, T, d, causal, out_dtype, s->sms, counter, make_ctl(s), cs));
+        launch_fwd_sm100(tm, rho != nullptr, y, lse, vexp, B, H, T, d, causal, out_dtype, s->sms, counter, make_ctl(s),
+                         cs));
 }
 
 size_t parallax_decode_workspace_bytes(int B, int H, int Tcap, int d) {

@@ -11,13 +11,24 @@
 //   S = Q K^T,  A = R K^T                       (bf16 x bf16 -> fp32, TMEM)
 //   O += P V,   M' += (P o A') V                (fp16 x fp16 -> fp32, TMEM)
 // with P = exp2(S log2e/sqrt(d) - m_ref) and A' = A / 256, both rounded to
-// fp16 and written back into TMEM as the A operands of the P.V UMMAs.  fp16 (not bf16) for these operands keeps the
-// rounding of P o A inside the error budget; the row sums l = sum P and
-// Abar' = sum P o A' are taken from the same rounded fp16 values the MMAs
-// consume, so the result is exact for the rounded weights.  The 1/256 factor
-// keeps P o A' finite for any |a| < 65504 while P may grow to 2^8 between
-// rescales (the running max is only moved when it rises by more than 8 in
-// log2 units; O and M are then rescaled in TMEM).
+// fp16 and written back into TMEM as the A operands of the P.V UMMAs.  fp16
+// (not bf16) for these operands keeps the rounding of P o A inside the error
+// budget; the row sums l = sum P and Abar' = sum P o A' are taken from the same
+// rounded fp16 values the MMAs consume, so the result is exact for the rounded
+// weights.  The running max is only moved when it rises by more than 8 in log2
+// units (O and M are then rescaled in TMEM), so P <= 2^8 between moves, and the
+// 1/256 on A keeps P o A' finite for |a| < 65504.
+//
+// V arrives as fp16 in blocks of 64 keys (one V stage), each scaled by its own
+// power of two 2^-e (convert.cu chooses e from the block's largest |v|, so V
+// keeps fp16 precision from about 1e-5 up to 2^23).  The stored P and P o A'
+// of that stage are multiplied by 2^e (exact in fp16's range), so P.V is
+// unchanged; the row sums are taken before that scaling.  Each softmax warp
+// reads its block's exponent (one byte) at the start of the tile.  (Folding
+// 2^e into the exponentials, or passing it through the V producer, put the
+// exponent on a critical path: measured 7-12% slower.)
+// An output that is still not finite (|v| >= 2^23, |a| >= 65504, non-finite
+// inputs) records PARALLAX_ERR_DEVICE_RANGE in the device error word.
 //
 // Why this shape (measured on B200): a tcgen05.mma costs at least ~45-50
 // cycles to issue, so UMMAs with N = 64 run at ~60% of the tensor rate while
@@ -32,6 +43,9 @@
 // a tile, then its A), P (the fp16 P and P o A' of a tile), O and M.  The
 // softmax releases X as soon as it has loaded S, and again once it has loaded
 // A; the P region is free once the previous tile's P.V UMMAs are done.
+// (Measured and dropped: a 768-thread layout with a separate epilogue
+// warpgroup, and converting V inside the kernel; both slowed the softmax
+// warps, which set the pace, more than they saved.)
 //
 // Roles (640 threads, one CTA per SM, persistent over (head, query tile)
 // items taken longest-first from an atomic work counter):
@@ -40,7 +54,7 @@
 //   warps 2..17     four softmax warpgroups; group g takes key columns
 //                   [32g, 32g+32) of every tile for all 128 rows, one row per
 //                   thread; the four exchange their partial row max through
-//                   shared memory and an mbarrier
+//                   shared memory and an mbarrier; then the item's epilogue
 //   warp 18 lane 0  issues the P.V UMMAs
 //   warp 19 lane 0  TMA for V (fp16, 64-key stages)
 // Every wait is a bounded mbarrier wait (no named barriers), so a wait that
@@ -60,7 +74,6 @@
 namespace plx {
 namespace {
 
-constexpr int D = 128;
 constexpr int BM = 128;                   // query rows per tile
 constexpr int BN = 128;                   // keys per tile
 constexpr int NGRP = 4;                   // softmax warpgroups
@@ -82,24 +95,30 @@ constexpr float A_SCALE = 1.0f / 256.0f;
 constexpr float A_UNSCALE = 256.0f;
 constexpr unsigned long long DRAIN_NS = 2000000ull;   // bound of the exit-time drain waits
 
-constexpr int Q_BYTES = BM * D * 2;       // 32 KB: two 64-column halves of [128 rows x 128 B]
-constexpr int K_BYTES = BN * D * 2;       // 32 KB: two halves of [128 keys x 128 B]
-constexpr int V_BYTES = VKEYS * D * 2;    // 16 KB fp16: two d-halves of [64 keys x 128 B]
-// shared-memory map (every tile region 1024-byte aligned)
-constexpr int OFF_Q = 0;
-constexpr int OFF_R = OFF_Q + Q_BYTES;
-constexpr int OFF_K = OFF_R + Q_BYTES;
-constexpr int OFF_V = OFF_K + KST * K_BYTES;
-constexpr int OFF_BARS = OFF_V + VST * V_BYTES;
+// Shared-memory map for head dim D (every tile region 1024-byte aligned).
+template <int D> struct Geo {
+    static constexpr int HALVES = D / 64;                // 128-byte (64-element) column blocks of a row
+    static constexpr int Q_BYTES = BM * D * 2;           // HALVES x [128 rows x 128 B]
+    static constexpr int K_BYTES = BN * D * 2;           // HALVES x [128 keys x 128 B]
+    static constexpr int V_BYTES = VKEYS * D * 2;        // fp16: HALVES x [64 keys x 128 B]
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_R = OFF_Q + Q_BYTES;
+    static constexpr int OFF_K = OFF_R + Q_BYTES;
+    static constexpr int OFF_V = OFF_K + KST * K_BYTES;
+    static constexpr int OFF_BARS = OFF_V + VST * V_BYTES;
+    static constexpr int OCOLS = D / NGRP;               // O/M columns each softmax group handles
+    static_assert(OCOLS % 16 == 0, "16-column TMEM loads");
+};
 
 // TMEM column map.  S(j) and then A(j) land in X.  Group g writes its fp16 P
-// (16 columns) and P o A' (16 columns) to [COL_P + 32g, +32).
+// (16 columns) and P o A' (16 columns) to [COL_P + 32g, +32).  O and M start
+// on 128-column boundaries for both head dims.
 constexpr uint32_t COL_X = 0, COL_P = 128, COL_O = 256, COL_M = 384;
 __host__ __device__ constexpr uint32_t col_p(uint32_t kk) { return COL_P + (kk >> 1) * GCOLS + (kk & 1) * 8; }
 constexpr uint32_t PA_SHIFT = GCOLS / 2;   // P o A' sits 16 columns after P
 
 constexpr uint32_t IDESC_S = idesc_f16(1, 1, 0, 0, BM, BN);     // bf16 Q/R (K-major) x bf16 K (K-major)
-constexpr uint32_t IDESC_PV = idesc_f16(0, 0, 0, 1, BM, D);     // f16 P (TMEM) x f16 V (MN-major)
+template <int D> constexpr uint32_t idesc_pv() { return idesc_f16(0, 0, 0, 1, BM, D); }   // f16 P (TMEM) x f16 V (MN-major)
 
 struct __align__(8) Bars {
     uint64_t qr_full, qr_empty;
@@ -121,8 +140,8 @@ struct __align__(8) Bars {
     float red_sum[2][NGRP][BM];   // [l or abar'][group][row] partial sums for the epilogue
 };
 
-constexpr size_t SMEM_BYTES = (size_t)OFF_BARS + sizeof(Bars);
-static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+template <int D> constexpr size_t smem_bytes() { return (size_t)Geo<D>::OFF_BARS + sizeof(Bars); }
+static_assert(smem_bytes<128>() <= 232448, "shared memory budget");
 
 struct Item {
     int bh, qt, nkv;
@@ -204,11 +223,13 @@ __device__ __forceinline__ void exp2_poly2(float &y0, float &y1, float x0, float
     y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
-template <bool WITH_RHO, typename Tout>
+template <int D, bool WITH_RHO, typename Tout>
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
           const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_v, Tout *__restrict__ y,
-          float *__restrict__ lse, int BH, int T, int causal, int *__restrict__ work_counter, DeviceCtl ctl) {
+          float *__restrict__ lse, const signed char *__restrict__ vexp_g, int BH, int T, int causal,
+          int *__restrict__ work_counter, DeviceCtl ctl) {
+    using Gm = Geo<D>;
     extern __shared__ __align__(1024) uint8_t smem[];
     // The swizzled tiles need a 1024-byte aligned base; there is no slack left
     // in the budget to realign, so refuse (recorded as a device error) if not.
@@ -216,7 +237,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (threadIdx.x == 0) atomicExch(ctl.err, PARALLAX_ERR_UNSUPPORTED);
         return;
     }
-    Bars *bars = reinterpret_cast<Bars *>(smem + OFF_BARS);
+    Bars *bars = reinterpret_cast<Bars *>(smem + Gm::OFF_BARS);
     const uint32_t sbase = smem_u32(smem);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -284,24 +305,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (!mbar_wait(smem_u32(&bars->qr_empty), (ic & 1) ^ 1, wc)) break;
             const uint32_t qf = smem_u32(&bars->qr_full);
             qr_armed = (int)(ic & 1);
-            mbar_arrive_expect_tx(qf, WITH_RHO ? 2 * Q_BYTES : Q_BYTES);
-            tma_load_3d(sbase + OFF_Q, &tm_q, qf, 0, q0, it.bh);
-            tma_load_3d(sbase + OFF_Q + Q_BYTES / 2, &tm_q, qf, 64, q0, it.bh);
-            if (WITH_RHO) {
-                tma_load_3d(sbase + OFF_R, &tm_r, qf, 0, q0, it.bh);
-                tma_load_3d(sbase + OFF_R + Q_BYTES / 2, &tm_r, qf, 64, q0, it.bh);
+            mbar_arrive_expect_tx(qf, WITH_RHO ? 2 * Gm::Q_BYTES : Gm::Q_BYTES);
+#pragma unroll
+            for (int h = 0; h < Gm::HALVES; ++h) {
+                tma_load_3d(sbase + Gm::OFF_Q + h * (Gm::Q_BYTES / Gm::HALVES), &tm_q, qf, h * 64, q0, it.bh);
+                if (WITH_RHO)
+                    tma_load_3d(sbase + Gm::OFF_R + h * (Gm::Q_BYTES / Gm::HALVES), &tm_r, qf, h * 64, q0, it.bh);
             }
             for (int j = 0; j < it.nkv; ++j, ++kc) {
                 const int s = kc % KST;
                 if (!mbar_wait(smem_u32(&bars->k_empty[s]), ((kc / KST) & 1) ^ 1, wc)) { ok = false; break; }
                 const uint32_t f = smem_u32(&bars->k_full[s]);
-                const uint32_t dst = sbase + OFF_K + s * K_BYTES;
+                const uint32_t dst = sbase + Gm::OFF_K + s * Gm::K_BYTES;
                 const bool skip = (ctl.debug_flags & DEBUG_FWD_SKIP_FIRST_K_LOAD) && kc == 0;
                 if (!skip) {
                     k_armed[s] = (int)((kc / KST) & 1);
-                    mbar_arrive_expect_tx(f, K_BYTES);
-                    tma_load_3d(dst, &tm_k, f, 0, j * BN, it.bh);
-                    tma_load_3d(dst + K_BYTES / 2, &tm_k, f, 64, j * BN, it.bh);
+                    mbar_arrive_expect_tx(f, Gm::K_BYTES);
+#pragma unroll
+                    for (int h = 0; h < Gm::HALVES; ++h)
+                        tma_load_3d(dst + h * (Gm::K_BYTES / Gm::HALVES), &tm_k, f, h * 64, j * BN, it.bh);
                 }
             }
         }
@@ -328,10 +350,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (!mbar_wait(smem_u32(&bars->v_empty[s]), ((vc / VST) & 1) ^ 1, wc)) { ok = false; break; }
                     const uint32_t f = smem_u32(&bars->v_full[s]);
                     v_armed[s] = (int)((vc / VST) & 1);
-                    const uint32_t dst = sbase + OFF_V + s * V_BYTES;
-                    mbar_arrive_expect_tx(f, V_BYTES);
-                    tma_load_3d(dst, &tm_v, f, 0, j * BN + vs * VKEYS, it.bh);
-                    tma_load_3d(dst + V_BYTES / 2, &tm_v, f, 64, j * BN + vs * VKEYS, it.bh);
+                    const uint32_t dst = sbase + Gm::OFF_V + s * Gm::V_BYTES;
+                    mbar_arrive_expect_tx(f, Gm::V_BYTES);
+#pragma unroll
+                    for (int h = 0; h < Gm::HALVES; ++h)
+                        tma_load_3d(dst + h * (Gm::V_BYTES / Gm::HALVES), &tm_v, f, h * 64, j * BN + vs * VKEYS,
+                                    it.bh);
                 }
             }
         }
@@ -346,14 +370,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // stream short.
         uint32_t kc = 0, G = 0;
         bool ok = true;
-        const uint64_t dq = sdesc_sw128(sbase + OFF_Q, 16, 1024);
-        const uint64_t dr = sdesc_sw128(sbase + OFF_R, 16, 1024);
-        const uint64_t dk = sdesc_sw128(sbase + OFF_K, 16, 1024);   // stage s: + s * K_BYTES / 16
+        const uint64_t dq = sdesc_sw128(sbase + Gm::OFF_Q, 16, 1024);
+        const uint64_t dr = sdesc_sw128(sbase + Gm::OFF_R, 16, 1024);
+        const uint64_t dk = sdesc_sw128(sbase + Gm::OFF_K, 16, 1024);   // stage s: + s * K_BYTES / 16
         auto issue_scores = [&](uint64_t da, uint64_t kd) {
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off = ((uint32_t)(kk >> 2) * (Q_BYTES / 2) + (uint32_t)(kk & 3) * 32) >> 4;
-                const uint32_t koff = ((uint32_t)(kk >> 2) * (K_BYTES / 2) + (uint32_t)(kk & 3) * 32) >> 4;
+                const uint32_t off = ((uint32_t)(kk >> 2) * (Gm::Q_BYTES / Gm::HALVES) + (uint32_t)(kk & 3) * 32) >> 4;
+                const uint32_t koff =
+                    ((uint32_t)(kk >> 2) * (Gm::K_BYTES / Gm::HALVES) + (uint32_t)(kk & 3) * 32) >> 4;
                 umma_ss(tmem + COL_X, da + off, kd + koff, IDESC_S, kk > 0 ? 1u : 0u);
             }
         };
@@ -372,7 +397,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     break;
                 }
                 tc_fence_after();
-                const uint64_t kd = dk + (uint64_t)(s * (K_BYTES >> 4));
+                const uint64_t kd = dk + (uint64_t)(s * (Gm::K_BYTES >> 4));
                 issue_scores(dq, kd);
                 tc_commit(smem_u32(&bars->s_full));
                 if constexpr (WITH_RHO) {
@@ -392,7 +417,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // ============================================== P.V UMMA issuer ==
         uint32_t vc = 0, G = 0;
         bool ok = true;
-        const uint64_t dv = sdesc_sw128(sbase + OFF_V, V_BYTES / 2, 1024);   // stage s: + s * V_BYTES / 16
+        constexpr uint32_t IDESC_PV = idesc_pv<D>();
+        const uint64_t dv = sdesc_sw128(sbase + Gm::OFF_V, Gm::V_BYTES / Gm::HALVES, 1024);   // + s * V_BYTES / 16
         for (uint32_t ic = 0; ok; ++ic) {
             int w;
             if (!next_item(bars, ic, w, wc)) break;
@@ -411,7 +437,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     const int s = vc % VST;
                     if (!mbar_wait(smem_u32(&bars->v_full[s]), (vc / VST) & 1, wc)) { ok = false; break; }
                     tc_fence_after();
-                    const uint64_t vd = dv + (uint64_t)(s * (V_BYTES >> 4));
+                    const uint64_t vd = dv + (uint64_t)(s * (Gm::V_BYTES >> 4));
 #pragma unroll
                     for (int k2 = 0; k2 < VKEYS / 16; ++k2) {
                         const int kk = vs * (VKEYS / 16) + k2;     // 16-key step within the tile
@@ -435,6 +461,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int r = quarter * 32 + lane;               // query row within the tile == TMEM lane
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const float scale_log2 = LOG2E / sqrtf((float)D);
+        const int vsg = (grp * GCOLS) / VKEYS;           // the V block (within a tile) of this group's keys
+        const int nblk = (T + VKEYS - 1) / VKEYS;        // 64-key V blocks per head, one exponent each
         uint32_t G = 0, ni = 0;   // key tiles and items processed by this CTA
         bool ok = true;
         for (uint32_t ic = 0; ok; ++ic) {
@@ -446,9 +474,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const Item it = item_of(w, BH, nq, T, causal);
             const int qrow = it.qt * BM + r;
             const int kvis = causal ? min(T, qrow + 1) : T;  // keys visible to this row
-            float m_ref = -INFINITY;
-            float l4[4] = {0.f, 0.f, 0.f, 0.f}, a4[4] = {0.f, 0.f, 0.f, 0.f};
+            float m_ref = -INFINITY, l = 0.f, ab = 0.f;
             for (int j = 0; j < it.nkv; ++j, ++G) {
+                // the exponent of this group's V block, needed only when P is stored
+                const int vblk = j * VPER + vsg;   // past the last block the keys read as zero
+                const int e = vblk < nblk ? (int)__ldg(vexp_g + (size_t)it.bh * nblk + vblk) : 0;
                 // ---- scores of this group's 32 keys, then release S ----
                 if (!warp_wait(smem_u32(&bars->s_full), G & 1, wc)) { ok = false; break; }
                 tc_fence_after();
@@ -489,16 +519,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (mx > m_ref + RESCALE_THRESHOLD) {
                     alpha = ex2(m_ref - mx);     // 0 when m_ref = -inf
                     m_ref = mx;
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        l4[i] *= alpha;
-                        a4[i] *= alpha;
-                    }
+                    l *= alpha;
+                    ab *= alpha;
                     moved = true;
                 }
                 // ---- P = exp2(z log2e - m_ref) as fp16, sums from the rounded values ----
                 const float neg_m = -m_ref;
                 uint32_t pk[GCOLS / 2];
+                float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int i = 0; i < GCOLS / 2; ++i) {
                     float x0, x1;
@@ -513,6 +541,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     pk[i] = pack_f16x2(e0, e1);
                     l4[i & 3] = add_f16x2_to_f32(l4[i & 3], pk[i]);
                 }
+                l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
                 uint32_t pak[WITH_RHO ? GCOLS / 2 : 1];
                 if constexpr (WITH_RHO) {
                     // ---- A of this group's 32 keys, then release X ----
@@ -526,6 +555,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(smem_u32(&bars->a_free));
+                    float a4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int i = 0; i < GCOLS / 2; ++i) {
                         float a0, a1;
@@ -533,6 +563,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         pak[i] = hmul2(pk[i], pack_f16x2(a0, a1));
                         a4[i & 3] = add_f16x2_to_f32(a4[i & 3], pak[i]);
                     }
+                    ab += (a4[0] + a4[1]) + (a4[2] + a4[3]);
                 }
                 // ---- the previous tile's P.V UMMAs are done: the P region is
                 // free and O, M' hold every earlier tile of this item ----
@@ -540,11 +571,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (!warp_wait(smem_u32(&bars->pv_done), (G - 1) & 1, wc)) { ok = false; break; }
                     tc_fence_after();
                 }
-                // a moved reference max rescales O and M' (each group its 32 columns)
+                // ---- V of this block holds v 2^-e: P and P o A' are stored as
+                // 2^e P and 2^e P o A', so the P.V products are unchanged (a
+                // power-of-two multiply is exact in fp16's range; e = 0 for
+                // ordinary magnitudes, and the branch is uniform in the warp) ----
+                {
+                    if (e != 0) {
+                        const __half2 two_e = __float2half2_rn(__int_as_float((127 + e) << 23));
+                        const uint32_t h2 = *reinterpret_cast<const uint32_t *>(&two_e);
+#pragma unroll
+                        for (int i = 0; i < GCOLS / 2; ++i) {
+                            pk[i] = hmul2(pk[i], h2);
+                            if constexpr (WITH_RHO) pak[i] = hmul2(pak[i], h2);
+                        }
+                    }
+                }
+                // a moved reference max rescales O and M' (each group d/4 columns)
                 if (__any_sync(0xffffffffu, moved && j > 0)) {
                     const float f = (moved && j > 0) ? alpha : 1.f;
 #pragma unroll 1
-                    for (int c = grp * GCOLS; c < grp * GCOLS + GCOLS; c += 16) {
+                    for (int c = grp * Gm::OCOLS; c < grp * Gm::OCOLS + Gm::OCOLS; c += 16) {
                         uint32_t t[16];
                         tmem_ld16(tmem + lane_off + COL_O + c, t);
                         tmem_wait_ld();
@@ -570,25 +616,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             if (!ok) break;
             // ---------------------------------------------- epilogue --
-            bars->red_sum[0][grp][r] = (l4[0] + l4[1]) + (l4[2] + l4[3]);
-            bars->red_sum[1][grp][r] = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+            bars->red_sum[0][grp][r] = l;
+            bars->red_sum[1][grp][r] = ab;
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&bars->esum));
             if (!warp_wait(smem_u32(&bars->esum), ni & 1, wc)) break;
             ++ni;
-            const float l = (bars->red_sum[0][0][r] + bars->red_sum[0][1][r]) +
-                            (bars->red_sum[0][2][r] + bars->red_sum[0][3][r]);
-            const float ab = (bars->red_sum[1][0][r] + bars->red_sum[1][1][r]) +
-                             (bars->red_sum[1][2][r] + bars->red_sum[1][3][r]);
+            const float lt = (bars->red_sum[0][0][r] + bars->red_sum[0][1][r]) +
+                             (bars->red_sum[0][2][r] + bars->red_sum[0][3][r]);
+            const float abt = (bars->red_sum[1][0][r] + bars->red_sum[1][1][r]) +
+                              (bars->red_sum[1][2][r] + bars->red_sum[1][3][r]);
             // the last P.V UMMAs of this item are done: O and M' are final
             if (!warp_wait(smem_u32(&bars->pv_done), (G - 1) & 1, wc)) break;
             tc_fence_after();
-            const float inv_l = 1.0f / l;
-            const float abar = ab * inv_l;
+            const float inv_l = 1.0f / lt;
+            const float abar = abt * inv_l;
             const bool store = qrow < T;
             Tout *yrow = y + ((size_t)it.bh * T + (store ? qrow : 0)) * D;
+            bool finite = true;
 #pragma unroll 1
-            for (int c = grp * GCOLS; c < grp * GCOLS + GCOLS; c += 16) {
+            for (int c = grp * Gm::OCOLS; c < grp * Gm::OCOLS + Gm::OCOLS; c += 16) {
                 uint32_t o[16], mm[16];
                 tmem_ld16(tmem + lane_off + COL_O + c, o);
                 if constexpr (WITH_RHO) tmem_ld16(tmem + lane_off + COL_M + c, mm);
@@ -603,6 +650,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     } else {
                         out[i] = ov;
                     }
+                    finite = finite && isfinite(out[i]);
                 }
                 if (store) {
                     if constexpr (sizeof(Tout) == 4) {
@@ -623,7 +671,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     }
                 }
             }
-            if (store && grp == 0 && lse != nullptr) lse[(size_t)it.bh * T + qrow] = (m_ref + log2f(l)) * LN2;
+            if (store && grp == 0 && lse != nullptr) lse[(size_t)it.bh * T + qrow] = (m_ref + log2f(lt)) * LN2;
+            // an output that is not finite: an input outside the kernel's range
+            if (__any_sync(0xffffffffu, store && !finite) && lane == 0) atomicCAS(ctl.err, 0, PARALLAX_ERR_DEVICE_RANGE);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&bars->om_free));
@@ -637,33 +687,42 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
 }
 
-template <bool WITH_RHO, typename Tout>
-cudaError_t launch_t(const FwdTensorMaps &tm, void *y, float *lse, int BH, int T, int causal, int sm_count,
-                     int *work_counter, const DeviceCtl &ctl, cudaStream_t s) {
+template <int D, bool WITH_RHO, typename Tout>
+cudaError_t launch_t(const FwdTensorMaps &tm, void *y, float *lse, const signed char *vexp, int BH, int T,
+                     int causal, int sm_count, int *work_counter, const DeviceCtl &ctl, cudaStream_t s) {
     static std::atomic<unsigned long long> limit_set{0};
-    if (cudaError_t e = ensure_smem_limit(k_fwd<WITH_RHO, Tout>, (int)SMEM_BYTES, limit_set)) return e;
+    auto kern = k_fwd<D, WITH_RHO, Tout>;
+    if (cudaError_t e = ensure_smem_limit(kern, (int)smem_bytes<D>(), limit_set)) return e;
     const int items = ((T + BM - 1) / BM) * BH;
     const int grid = items < sm_count ? items : sm_count;
     cudaError_t e = cudaMemsetAsync(work_counter, 0, sizeof(int), s);
     if (e != cudaSuccess) return e;
-    k_fwd<WITH_RHO, Tout><<<grid, NTHREADS, SMEM_BYTES, s>>>(tm.q, tm.k, tm.r, tm.v16, static_cast<Tout *>(y), lse,
-                                                             BH, T, causal, work_counter, ctl);
+    kern<<<grid, NTHREADS, smem_bytes<D>(), s>>>(tm.q, tm.k, tm.r, tm.v, static_cast<Tout *>(y), lse, vexp, BH, T,
+                                                 causal, work_counter, ctl);
     return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_d(const FwdTensorMaps &tm, bool with_rho, void *y, float *lse, const signed char *vexp, int BH,
+                     int T, int causal, int out_dtype, int sm_count, int *work_counter, const DeviceCtl &ctl,
+                     cudaStream_t s) {
+    if (out_dtype == PARALLAX_F32) {
+        if (with_rho) return launch_t<D, true, float>(tm, y, lse, vexp, BH, T, causal, sm_count, work_counter, ctl, s);
+        return launch_t<D, false, float>(tm, y, lse, vexp, BH, T, causal, sm_count, work_counter, ctl, s);
+    }
+    if (with_rho)
+        return launch_t<D, true, __nv_bfloat16>(tm, y, lse, vexp, BH, T, causal, sm_count, work_counter, ctl, s);
+    return launch_t<D, false, __nv_bfloat16>(tm, y, lse, vexp, BH, T, causal, sm_count, work_counter, ctl, s);
 }
 
 }  // namespace
 
-cudaError_t launch_fwd_sm100(const FwdTensorMaps &tm, bool with_rho, void *y, float *lse, int B, int H, int T,
-                             int d, int causal, int out_dtype, int sm_count, int *work_counter, const DeviceCtl &ctl,
-                             cudaStream_t s) {
-    (void)d;
+cudaError_t launch_fwd_sm100(const FwdTensorMaps &tm, bool with_rho, void *y, float *lse, const signed char *vexp,
+                             int B, int H, int T, int d, int causal, int out_dtype, int sm_count, int *work_counter,
+                             const DeviceCtl &ctl, cudaStream_t s) {
     const int BH = B * H;
-    if (out_dtype == PARALLAX_F32) {
-        if (with_rho) return launch_t<true, float>(tm, y, lse, BH, T, causal, sm_count, work_counter, ctl, s);
-        return launch_t<false, float>(tm, y, lse, BH, T, causal, sm_count, work_counter, ctl, s);
-    }
-    if (with_rho) return launch_t<true, __nv_bfloat16>(tm, y, lse, BH, T, causal, sm_count, work_counter, ctl, s);
-    return launch_t<false, __nv_bfloat16>(tm, y, lse, BH, T, causal, sm_count, work_counter, ctl, s);
+    if (d == 64) return launch_d<64>(tm, with_rho, y, lse, vexp, BH, T, causal, out_dtype, sm_count, work_counter, ctl, s);
+    return launch_d<128>(tm, with_rho, y, lse, vexp, BH, T, causal, out_dtype, sm_count, work_counter, ctl, s);
 }
 
 }  // namespace plx

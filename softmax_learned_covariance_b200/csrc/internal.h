@@ -34,9 +34,6 @@ struct DeviceCtl {
 };
 constexpr unsigned DEBUG_FWD_SKIP_FIRST_K_LOAD = 1u;   // fwd: never load the first K tile
 
-// V [rows, d] bf16 -> fp16 (the PV operand precision of the tensor-core forward)
-cudaError_t launch_convert_bf16_to_f16(const void *src, void *dst, size_t n, cudaStream_t s);
-
 // fp32 / bf16 CUDA-core forward (one warp per query row)
 cudaError_t launch_fwd_simt(const void *q, const void *k, const void *v, const void *rho, void *y, float *lse,
                             int B, int H, int T, int d, int causal, int in_dtype, int out_dtype, cudaStream_t s);
@@ -74,14 +71,21 @@ int *noalloc_error_word();
 cudaError_t launch_rho_proj(const CUtensorMap &tm_x, const CUtensorMap &tm_w, void *rho, int B, int T, int d_model,
                             int H, int d, int sm_count, const DeviceCtl &ctl, cudaStream_t s);
 
-// tcgen05 causal/full prefill forward, bf16 in, fp16 V copy, fp32 accumulate
+// V [B*H, T, d] bf16 -> fp16 in 64-key blocks, block b of head bh scaled by
+// 2^-vexp[bh * v16_blocks(T) + b] (the forward kernel's P.V operand).
+int v16_blocks(int T);
+cudaError_t launch_v_to_f16_blocks(const void *v, void *v16, signed char *vexp, int BH, int T, int d,
+                                   cudaStream_t s);
+
+// tcgen05 causal/full prefill forward: bf16 q, k, rho, fp16 block-scaled V
+// (tensor map `v` over the output of launch_v_to_f16_blocks, exponents in
+// `vexp`), fp32 accumulation, d in {64, 128}.  work_counter: one device int,
+// reset by the launch (stream-ordered), the persistent grid's item counter.
 struct FwdTensorMaps {
-    CUtensorMap q, k, r, v16;
+    CUtensorMap q, k, r, v;
 };
-// work_counter: one device int, reset by the launch (stream-ordered) and used as the
-// persistent grid's atomic item counter.
-cudaError_t launch_fwd_sm100(const FwdTensorMaps &tm, bool with_rho, void *y, float *lse, int B, int H, int T,
-                             int d, int causal, int out_dtype, int sm_count, int *work_counter, const DeviceCtl &ctl,
-                             cudaStream_t s);
+cudaError_t launch_fwd_sm100(const FwdTensorMaps &tm, bool with_rho, void *y, float *lse, const signed char *vexp,
+                             int B, int H, int T, int d, int causal, int out_dtype, int sm_count, int *work_counter,
+                             const DeviceCtl &ctl, cudaStream_t s);
 
 }  // namespace plx

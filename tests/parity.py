@@ -3,6 +3,15 @@
 Tolerances for the bf16 tensor-core path: per head, max abs error <= 2e-2 and
 relative Frobenius error ||y - y_ref||_F / ||y_ref||_F <= 5e-3, gated on the
 fp32 output; fp32 path: max abs error <= 1e-4.  lse: max abs error <= 1e-3.
+
+The 2e-2 absolute bound is stated for the workloads' value scales (unit
+normal q, k, v; probe rho with standard deviation 0.905).  The operator is
+linear in V, and its rounding error on the correction term grows in
+proportion to the probe (the 16-bit weights P o (k . rho) carry a fixed
+relative error), so for inputs with V scaled by s_v or rho scaled by
+s_rho / 0.905 the absolute bound scales by the same factor
+(``assert_bf16_parity_scaled``); the relative Frobenius bound is scale-free
+and stays 5e-3.
 """
 from __future__ import annotations
 
@@ -31,6 +40,16 @@ def assert_bf16_parity(y, ref, head_axes=2, what=""):
     assert np.all(np.isfinite(y)), f"{what}: non-finite output"
     ma, rf = head_errors(y, ref, head_axes)
     assert ma.max() <= BF16_MAX_ABS, f"{what}: worst head max abs {ma.max():.3e} > {BF16_MAX_ABS}"
+    assert rf.max() <= BF16_REL_F, f"{what}: worst head rel-F {rf.max():.3e} > {BF16_REL_F}"
+    return float(ma.max()), float(rf.max())
+
+
+def assert_bf16_parity_scaled(y, ref, head_axes, scale, what=""):
+    """bf16 gates for inputs scaled away from the workloads' value scales: the
+    max-abs bound times ``scale``, the relative Frobenius bound unchanged."""
+    assert np.all(np.isfinite(y)), f"{what}: non-finite output"
+    ma, rf = head_errors(y, ref, head_axes)
+    assert ma.max() <= BF16_MAX_ABS * scale, f"{what}: worst head max abs {ma.max():.3e} > {BF16_MAX_ABS * scale:.3e}"
     assert rf.max() <= BF16_REL_F, f"{what}: worst head rel-F {rf.max():.3e} > {BF16_REL_F}"
     return float(ma.max()), float(rf.max())
 

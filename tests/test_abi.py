@@ -38,7 +38,7 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_strerror_covers_all_codes(L):
-    for code in range(9):
+    for code in range(10):
         s = plx.parallax_strerror(code)
         assert s and s != "unknown status"
     assert plx.parallax_strerror(99) == "unknown status"
@@ -64,7 +64,7 @@ def test_fwd_host_validation(L):
     assert fwd(L, lse=P(0x10002)) == 3
     assert fwd(L, i=1, o=5) == 4
     assert fwd(L, i=0, o=1) == 4
-    assert fwd(L, d=64, i=1, o=0) == 5      # bf16 tensor-core path needs d = 128
+    assert fwd(L, d=32, i=1, o=0) == 2      # head dims 64 and 128 only
 
 
 def test_decode_host_validation(L):
