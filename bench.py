@@ -427,7 +427,8 @@ def run_ours(args, rank, world):
         e2e_pre = {"value": whole_job_rate(p_flops + r_flops, e_ms / ksteps, world) / 1e12, "unit": "TFLOP/s",
                    "h2d_bytes_per_step": h2d_p, "d2h_bytes_per_step": yp.numel() * 4, "steps": ksteps}
 
-    extras = measure_extras(args, stream, barrier, world, peaks, pc, dpq, dpk, dpv, yp, lp, fwd_ms)
+    extras = measure_extras(args, stream, barrier, world, peaks, pc, dpq, dpk, dpv, yp, lp, fwd_ms, dx, dw,
+                            rp_ms + fwd_ms)
     decode_long = None if args.no_decode_long else measure_decode_long(args, peaks)
 
     dec_tbs = whole_job_rate(d_bytes, dec_ms, world) / 1e12
@@ -450,8 +451,8 @@ def run_ours(args, rank, world):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) q,k,v; rho ~ N(0,0.05^2) for decode; x ~ N(0,1), W_R ~ N(0,0.02^2) for prefill)",
-        "config": {"workload": "decode step B=64 H=16 d=128 ctx=4096 (headline) + prefill B=8 T=%d H=16 d=128 "
-                               "d_model=2048 causal" % pc["T"],
+        "config": {"workload": "decode step B=64 H=16 d=128 ctx=4096 (headline) + prefill B=%d T=%d H=16 d=128 "
+                               "d_model=2048 causal" % (pc["B"], pc["T"]),
                    "decode": dict(DECODE_CFG), "prefill": dict(pc), "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (2.1 GB decode cache, 0.6 GB prefill tensors); no flush"},
         "roofline": {"bound": "hbm", "kernel": "parallax_decode (split + combine)", "achieved": round(dec_tbs * 1e3 / world, 1),
@@ -470,6 +471,7 @@ def run_ours(args, rank, world):
         "e2e": e2e,
         "decode_paged": extras["decode_paged"],
         "softmax_only_fwd": extras["softmax_only_fwd"],
+        "fwd_fused": extras["fwd_fused"],
         "decode_long": decode_long,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
@@ -481,10 +483,12 @@ def run_ours(args, rank, world):
 PAGED_CFG = dict(B=64, Hq=32, Hkv=8, page_size=64, ctx=4096, d=128)
 
 
-def measure_extras(args, stream, barrier, world, peaks, pc, dpq, dpk, dpv, yp, lp, fwd_ms):
+def measure_extras(args, stream, barrier, world, peaks, pc, dpq, dpk, dpv, yp, lp, fwd_ms, dx, dw, pipe_ms):
     """Measurements beside the step (not part of it, not in its timed region):
-    the paged grouped-head decode, and the softmax-only instantiation of the
-    prefill on the same inputs (the compute-matched reference point)."""
+    the paged grouped-head decode, the softmax-only instantiation of the
+    prefill on the same inputs (the compute-matched reference point), and the
+    prefill with the probe computed inside the kernel (parallax_fwd_fused)
+    against the two-launch pipeline rho_proj + fwd."""
     import torch
 
     import softmax_learned_covariance_b200 as plx
@@ -541,7 +545,16 @@ def measure_extras(args, stream, barrier, world, peaks, pc, dpq, dpk, dpv, yp, l
     smx = {"ms": round(s_ms, 4), "tflops": round(s_tf, 2), "flops": 4 * pc["d"] * pairs,
            "parallax_over_softmax_time": round(fwd_ms / s_ms, 3),
            "note": "rho = NULL instantiation of the same kernel (2 of the 4 GEMMs); same inputs and shape"}
-    return {"decode_paged": paged, "softmax_only_fwd": smx}
+    # ---- probe rho = x W_R inside the prefill kernel ----
+    with torch.cuda.stream(stream):
+        f_ms = timed(lambda: plx.parallax_fwd_fused(dpq, dpk, dpv, dx, dw, y=yp, lse=lp, stream=stream), args.steps)
+    f_flops = prefill_flops(pc["B"], pc["H"], pc["T"], pc["d"]) + rho_proj_flops(pc["B"], pc["T"], pc["d_model"],
+                                                                                 pc["H"], pc["d"])
+    fused = {"ms": round(f_ms, 4), "tflops": round(f_flops / (f_ms * 1e-3) / 1e12, 2), "flops": f_flops,
+             "two_launch_ms": round(pipe_ms, 4), "speedup_vs_two_launch": round(pipe_ms / f_ms, 3),
+             "note": "parallax_fwd_fused (rho computed per query tile in the kernel, never in HBM) vs "
+                     "parallax_rho_proj + parallax_fwd on the same inputs; flops count both GEMM families"}
+    return {"decode_paged": paged, "softmax_only_fwd": smx, "fwd_fused": fused}
 
 
 # --------------------------------------------------------------------------- #

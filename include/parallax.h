@@ -114,6 +114,28 @@ PARALLAX_API int parallax_fwd(const void *q, const void *k, const void *v, const
                  int in_dtype, int out_dtype, parallax_stream_t stream);
 
 /*
+ * parallax_fwd_fused -- parallax_fwd with the probe computed inside the kernel.
+ *
+ * Passage: encorp.ai blog, section "Por que eliminar el solucionador de
+ * gradiente conjugado..." (the probe comes from a learned projector W_R of the
+ * layer input), zubnet.ai news item on Parallax, paragraph 2 (rho_i = W_R x_i).
+ * Instead of reading rho from memory, each 128-row query tile of a head
+ * computes its probe tile rho = x[b, rows, :] W_R[:, h*d:(h+1)*d] on the tensor
+ * cores (fp32 accumulation over d_model, rounded to bf16 as parallax_rho_proj
+ * rounds it) and keeps it on chip; rho never goes to HBM.
+ *
+ *   q, k, v : [B, H, T, d] bf16;  x : [B, T, d_model] bf16 (the layer input);
+ *   W_R     : [d_model, H*d] bf16 row-major (column block h is head h).
+ *   y, lse, causal, out_dtype: as parallax_fwd.
+ *   d == 128 (PARALLAX_ERR_UNSUPPORTED otherwise); d_model a multiple of 64.
+ *   in_dtype must be BF16.  Scratch as parallax_fwd.
+ * With W_R = 0 the result is bitwise the softmax-only result of parallax_fwd.
+ */
+PARALLAX_API int parallax_fwd_fused(const void *q, const void *k, const void *v, const void *x, const void *W_R,
+                                    void *y, float *lse, int B, int H, int T, int d, int d_model, int causal,
+                                    int in_dtype, int out_dtype, parallax_stream_t stream);
+
+/*
  * parallax_decode -- one new query token per sequence against a KV cache.
  *
  * Passage: zubnet.ai news item on Parallax, paragraph 2 (the KV cache is still

@@ -11,6 +11,7 @@ library is missing or a call fails, a ``ParallaxError`` is raised.
 
 Functions keep the C names:
     parallax_fwd(q, k, v, rho=None, causal=True, out_dtype=torch.float32) -> (y, lse)
+    parallax_fwd_fused(q, k, v, x, W_R, causal=True) -> (y, lse)     probe rho = x W_R in the kernel
     parallax_decode(q, rho, kcache, vcache, seqlens, out_dtype=torch.float32) -> (y, lse)
     parallax_decode_ex(..., workspace) -> (y, lse)          caller-owned split scratch
     parallax_decode_paged(q, rho, kpages, vpages, block_table, seqlens) -> (y, lse)
@@ -24,7 +25,7 @@ import os
 import threading
 
 __all__ = [
-    "ParallaxError", "lib", "parallax_fwd", "parallax_decode", "parallax_decode_ex", "parallax_decode_paged",
+    "ParallaxError", "lib", "parallax_fwd", "parallax_fwd_fused", "parallax_decode", "parallax_decode_ex", "parallax_decode_paged",
     "parallax_rho_proj", "parallax_decode_workspace_bytes", "parallax_last_device_error",
     "parallax_strerror", "parallax_device_sm_count", "LIB_PATH", "F32", "BF16",
 ]
@@ -52,6 +53,7 @@ def lib() -> ctypes.CDLL:
             L = ctypes.CDLL(LIB_PATH)
             P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
             L.parallax_fwd.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, P]
+            L.parallax_fwd_fused.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P]
             L.parallax_decode.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, P]
             L.parallax_decode_ex.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, P, S, P]
             L.parallax_decode_paged.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, P]
@@ -62,7 +64,7 @@ def lib() -> ctypes.CDLL:
             L.parallax_strerror.restype = ctypes.c_char_p
             L.parallax_last_device_error.argtypes = [P]
             L.parallax_device_sm_count.argtypes = []
-            for f in (L.parallax_fwd, L.parallax_decode, L.parallax_decode_ex, L.parallax_decode_paged,
+            for f in (L.parallax_fwd, L.parallax_fwd_fused, L.parallax_decode, L.parallax_decode_ex, L.parallax_decode_paged,
                       L.parallax_rho_proj,
                       L.parallax_last_device_error, L.parallax_device_sm_count):
                 f.restype = I
@@ -133,6 +135,29 @@ def parallax_fwd(q, k, v, rho=None, causal: bool = True, out_dtype=None, y=None,
     st = lib().parallax_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(rho), _ptr(y), _ptr(lse), B, H, T, d,
                             int(bool(causal)), _dtype_code(q.dtype), _dtype_code(y.dtype), _stream(stream))
     _check(st, "parallax_fwd")
+    return y, lse
+
+
+def parallax_fwd_fused(q, k, v, x, W_R, causal: bool = True, out_dtype=None, y=None, lse=None, stream=None,
+                       want_lse: bool = True):
+    """Prefill with the probe rho = x W_R computed in the kernel.
+
+    q, k, v: [B, H, T, d] bf16 (d = 128); x: [B, T, d_model] bf16; W_R: [d_model, H*d] bf16.
+    """
+    torch = _torch()
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (x, "x"), (W_R, "W_R")):
+        _need(t, n)
+    B, H, T, d = q.shape
+    d_model = x.shape[-1]
+    out_dtype = out_dtype or torch.float32
+    if y is None:
+        y = torch.empty((B, H, T, d), dtype=out_dtype, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
+    st = lib().parallax_fwd_fused(_ptr(q), _ptr(k), _ptr(v), _ptr(x), _ptr(W_R), _ptr(y), _ptr(lse), B, H, T, d,
+                                  d_model, int(bool(causal)), _dtype_code(q.dtype), _dtype_code(y.dtype),
+                                  _stream(stream))
+    _check(st, "parallax_fwd_fused")
     return y, lse
 
 

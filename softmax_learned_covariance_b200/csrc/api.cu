@@ -153,6 +153,31 @@ int encode(CUtensorMap *m, CUtensorMapDataType dt, const void *base, int rank, c
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
+// Common part of the tensor-core prefill calls: per-call scratch (the work
+// counter, the block exponents of V and V as block-scaled fp16), the
+// conversion of V, and the tensor maps of q, k and the fp16 V.  tm->r, tm->x
+// and tm->w are set to a valid map the caller replaces when it needs them.
+int prepare_fwd(const void *q, const void *k, const void *v, int B, int H, int T, int d, cudaStream_t cs,
+                CallScratch &scratch, FwdTensorMaps *tm, signed char **vexp, int **counter) {
+    const size_t n = (size_t)B * H * T * d;
+    const size_t nexp = ((size_t)B * H * v16_blocks(T) + 255) & ~(size_t)255;
+    void *ws = nullptr;
+    int st;
+    if ((st = scratch.get(256 + nexp + n * 2, &ws))) return st;
+    *counter = static_cast<int *>(ws);
+    *vexp = static_cast<signed char *>(ws) + 256;
+    void *v16 = static_cast<char *>(ws) + 256 + nexp;
+    if (launch_v_to_f16_blocks(v, v16, *vexp, B * H, T, d, cs) != cudaSuccess) return PARALLAX_ERR_CUDA;
+    const uint64_t dims[3] = {(uint64_t)d, (uint64_t)T, (uint64_t)B * H};
+    // boxes: 64 head-dim columns (128 B, the swizzle span) x {128 query rows, 128 keys, 64 keys}
+    const uint32_t box_q[3] = {64, 128, 1}, box_k[3] = {64, 128, 1}, box_v[3] = {64, 64, 1};
+    if ((st = encode(&tm->q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, 3, dims, box_q, 2))) return st;
+    if ((st = encode(&tm->k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k, 3, dims, box_k, 2))) return st;
+    if ((st = encode(&tm->v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, v16, 3, dims, box_v, 2))) return st;
+    tm->r = tm->x = tm->w = tm->q;
+    return PARALLAX_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -216,34 +241,55 @@ int parallax_fwd(const void *q, const void *k, const void *v, const void *rho, v
     if (f32) return status_of(launch_fwd_simt(q, k, v, rho, y, lse, B, H, T, d, causal, in_dtype, out_dtype, cs));
 
     if ((st = ensure_encoder())) return st;
-    // scratch: the persistent grid's work counter, the block exponents of V,
-    // and V as block-scaled fp16
-    const size_t n = (size_t)B * H * T * d;
-    const size_t nexp = ((size_t)B * H * v16_blocks(T) + 255) & ~(size_t)255;
     CallScratch scratch(s, cs);
-    void *ws = nullptr;
-    if ((st = scratch.get(256 + nexp + n * 2, &ws))) return st;
-    int *counter = static_cast<int *>(ws);
-    signed char *vexp = static_cast<signed char *>(ws) + 256;
-    void *v16 = static_cast<char *>(ws) + 256 + nexp;
-    if (launch_v_to_f16_blocks(v, v16, vexp, B * H, T, d, cs) != cudaSuccess) return PARALLAX_ERR_CUDA;
-
     FwdTensorMaps tm;
-    const uint64_t dims[3] = {(uint64_t)d, (uint64_t)T, (uint64_t)B * H};
-    // boxes: 64 head-dim columns (128 B, the swizzle span) x {128 query rows, 128 keys, 64 keys}
-    const uint32_t box_q[3] = {64, 128, 1}, box_k[3] = {64, 128, 1}, box_v[3] = {64, 64, 1};
-    if ((st = encode(&tm.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, 3, dims, box_q, 2))) return st;
-    if ((st = encode(&tm.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k, 3, dims, box_k, 2))) return st;
-    if ((st = encode(&tm.v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, v16, 3, dims, box_v, 2))) return st;
-
+    signed char *vexp = nullptr;
+    int *counter = nullptr;
+    if ((st = prepare_fwd(q, k, v, B, H, T, d, cs, scratch, &tm, &vexp, &counter))) return st;
     if (rho) {
+        const uint64_t dims[3] = {(uint64_t)d, (uint64_t)T, (uint64_t)B * H};
+        const uint32_t box_q[3] = {64, 128, 1};
         if ((st = encode(&tm.r, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rho, 3, dims, box_q, 2))) return st;
-    } else {
-        tm.r = tm.q;
     }
     return status_of(
         launch_fwd_sm100(tm, rho != nullptr, y, lse, vexp, B, H, T, d, causal, out_dtype, s->sms, counter, make_ctl(s),
                          cs));
+}
+
+int parallax_fwd_fused(const void *q, const void *k, const void *v, const void *x, const void *W_R, void *y,
+                       float *lse, int B, int H, int T, int d, int d_model, int causal, int in_dtype, int out_dtype,
+                       parallax_stream_t stream) {
+    if (!q || !k || !v || !x || !W_R || !y) return PARALLAX_ERR_NULL;
+    if (B < 1 || H < 1 || T < 1 || (d != 64 && d != 128) || d_model < 64 || d_model % 64 != 0)
+        return PARALLAX_ERR_SHAPE;
+    if ((long long)B * H * T * d > (1ll << 40) || (long long)B * H > (1ll << 30) || (long long)B * T > (1ll << 31) - 1 ||
+        (long long)d_model * H * d > (1ll << 40))
+        return PARALLAX_ERR_SHAPE;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(x) || !aligned16(W_R) || !aligned16(y) ||
+        (lse && !aligned4(lse)))
+        return PARALLAX_ERR_ALIGN;
+    if (in_dtype != PARALLAX_BF16 || (out_dtype != PARALLAX_F32 && out_dtype != PARALLAX_BF16))
+        return PARALLAX_ERR_DTYPE;
+    if (d != 128) return PARALLAX_ERR_UNSUPPORTED;
+    DevState *s = nullptr;
+    int st = get_state(&s);
+    if (st) return st;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if ((st = ensure_encoder())) return st;
+    CallScratch scratch(s, cs);
+    FwdTensorMaps tm;
+    signed char *vexp = nullptr;
+    int *counter = nullptr;
+    if ((st = prepare_fwd(q, k, v, B, H, T, d, cs, scratch, &tm, &vexp, &counter))) return st;
+    // x as [B*T, d_model] in boxes of 64 x 128 rows; W_R as [d_model, H*d] in boxes of 64 x 64
+    const uint64_t dx[2] = {(uint64_t)d_model, (uint64_t)B * T};
+    const uint32_t bx[2] = {64, 128};
+    const uint64_t dw[2] = {(uint64_t)H * d, (uint64_t)d_model};
+    const uint32_t bw[2] = {64, 64};
+    if ((st = encode(&tm.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, 2, dx, bx, 2))) return st;
+    if ((st = encode(&tm.w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W_R, 2, dw, bw, 2))) return st;
+    return status_of(launch_fwd_fused_sm100(tm, y, lse, vexp, B, H, T, d_model, causal, out_dtype, s->sms, counter,
+                                            make_ctl(s), cs));
 }
 
 size_t parallax_decode_workspace_bytes(int B, int H, int Tcap, int d) {

@@ -122,6 +122,7 @@ template <int D> constexpr uint32_t idesc_pv() { return idesc_f16(0, 0, 0, 1, BM
 
 struct __align__(8) Bars {
     uint64_t qr_full, qr_empty;
+    uint64_t r_tmem, r_smem;      // fused probe: R = X W_R in TMEM; R converted into shared memory
     uint64_t k_full[KST], k_empty[KST];
     uint64_t v_full[VST], v_empty[VST];
     uint64_t s_full, a_full;      // S, A UMMAs of the current tile done
@@ -223,13 +224,20 @@ __device__ __forceinline__ void exp2_poly2(float &y0, float &y1, float x0, float
     y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
-template <int D, bool WITH_RHO, typename Tout>
+template <int D, bool WITH_RHO, bool FUSED, typename Tout>
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-          const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_v, Tout *__restrict__ y,
-          float *__restrict__ lse, const signed char *__restrict__ vexp_g, int BH, int T, int causal,
-          int *__restrict__ work_counter, DeviceCtl ctl) {
+          const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_v,
+          const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w, Tout *__restrict__ y,
+          float *__restrict__ lse, const signed char *__restrict__ vexp_g, int BH, int H, int T, int d_model,
+          int causal, int *__restrict__ work_counter, DeviceCtl ctl) {
     using Gm = Geo<D>;
+    static_assert(!FUSED || (WITH_RHO && D == 128), "the fused probe needs the correction branch and d = 128");
+    // fused probe: X W_R is accumulated over d_model in chunks of 64 that
+    // stream through the K ring (X chunk [128 rows x 64], W_R chunk [64 x d])
+    constexpr int XC_BYTES = BM * 64 * 2, WC_BYTES = 64 * D * 2;
+    static_assert(!FUSED || XC_BYTES + WC_BYTES <= Gm::K_BYTES, "an X / W_R chunk fits a K stage");
+    const int nchunk = FUSED ? d_model / 64 : 0;
     extern __shared__ __align__(1024) uint8_t smem[];
     // The swizzled tiles need a 1024-byte aligned base; there is no slack left
     // in the budget to realign, so refuse (recorded as a device error) if not.
@@ -244,6 +252,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (threadIdx.x == 0) {
         mbar_init(smem_u32(&bars->qr_full), 1);
         mbar_init(smem_u32(&bars->qr_empty), 1);
+        mbar_init(smem_u32(&bars->r_tmem), 1);
+        mbar_init(smem_u32(&bars->r_smem), NSOFT_WARPS);
         for (int s = 0; s < KST; ++s) {
             mbar_init(smem_u32(&bars->k_full[s]), 1);
             mbar_init(smem_u32(&bars->k_empty[s]), 1);
@@ -288,7 +298,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // ===================================== scheduler + Q/R/K producer ==
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
-        if (WITH_RHO) tma_prefetch_desc(&tm_r);
+        if (WITH_RHO && !FUSED) tma_prefetch_desc(&tm_r);
+        if (FUSED) {
+            tma_prefetch_desc(&tm_x);
+            tma_prefetch_desc(&tm_w);
+        }
         uint32_t kc = 0;
         int k_armed[KST], qr_armed = -1;   // parity of each buffer's last fill still to land, -1 if none
         for (int s = 0; s < KST; ++s) k_armed[s] = -1;
@@ -305,12 +319,31 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (!mbar_wait(smem_u32(&bars->qr_empty), (ic & 1) ^ 1, wc)) break;
             const uint32_t qf = smem_u32(&bars->qr_full);
             qr_armed = (int)(ic & 1);
-            mbar_arrive_expect_tx(qf, WITH_RHO ? 2 * Gm::Q_BYTES : Gm::Q_BYTES);
+            mbar_arrive_expect_tx(qf, (WITH_RHO && !FUSED) ? 2 * Gm::Q_BYTES : Gm::Q_BYTES);
 #pragma unroll
             for (int h = 0; h < Gm::HALVES; ++h) {
                 tma_load_3d(sbase + Gm::OFF_Q + h * (Gm::Q_BYTES / Gm::HALVES), &tm_q, qf, h * 64, q0, it.bh);
-                if (WITH_RHO)
+                if (WITH_RHO && !FUSED)
                     tma_load_3d(sbase + Gm::OFF_R + h * (Gm::Q_BYTES / Gm::HALVES), &tm_r, qf, h * 64, q0, it.bh);
+            }
+            if constexpr (FUSED) {
+                // X rows of this query tile (row b*T + t of x) and head h's
+                // columns of W_R, 64 of d_model at a time, through the K ring
+                const int xrow = (it.bh / H) * T + q0, wcol = (it.bh % H) * D;
+                for (int c = 0; c < nchunk && ok; ++c, ++kc) {
+                    const int s = kc % KST;
+                    if (!mbar_wait(smem_u32(&bars->k_empty[s]), ((kc / KST) & 1) ^ 1, wc)) { ok = false; break; }
+                    const uint32_t f = smem_u32(&bars->k_full[s]);
+                    const uint32_t dst = sbase + Gm::OFF_K + s * Gm::K_BYTES;
+                    if ((ctl.debug_flags & DEBUG_FWD_SKIP_FIRST_K_LOAD) && kc == 0) continue;
+                    k_armed[s] = (int)((kc / KST) & 1);
+                    mbar_arrive_expect_tx(f, XC_BYTES + WC_BYTES);
+                    tma_load_2d(dst, &tm_x, f, c * 64, xrow);
+#pragma unroll
+                    for (int h = 0; h < Gm::HALVES; ++h)
+                        tma_load_2d(dst + XC_BYTES + h * (64 * 64 * 2), &tm_w, f, wcol + h * 64, c * 64);
+                }
+                if (!ok) break;
             }
             for (int j = 0; j < it.nkv; ++j, ++kc) {
                 const int s = kc % KST;
@@ -373,6 +406,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint64_t dq = sdesc_sw128(sbase + Gm::OFF_Q, 16, 1024);
         const uint64_t dr = sdesc_sw128(sbase + Gm::OFF_R, 16, 1024);
         const uint64_t dk = sdesc_sw128(sbase + Gm::OFF_K, 16, 1024);   // stage s: + s * K_BYTES / 16
+        // fused probe: R[128 x d] += X chunk (K-major) x W_R chunk (MN-major) into the P region
+        constexpr uint32_t IDESC_R = idesc_f16(1, 1, 0, 1, BM, D);
+        auto issue_probe_chunk = [&](uint32_t stage_addr, bool first) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t adesc = sdesc_sw128(stage_addr + kk * 32, 16, 1024);
+                const uint64_t bdesc = sdesc_sw128(stage_addr + XC_BYTES + kk * 16 * 128, 64 * 128, 1024);
+                umma_ss(tmem + COL_P, adesc, bdesc, IDESC_R, (first && kk == 0) ? 0u : 1u);
+            }
+        };
         auto issue_scores = [&](uint64_t da, uint64_t kd) {
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
@@ -389,6 +432,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (w >= items) break;
             const Item it = item_of(w, BH, nq, T, causal);
             if (!mbar_wait(smem_u32(&bars->qr_full), ic & 1, wc)) break;
+            if constexpr (FUSED) {
+                // R of this item into the P region once the last P.V UMMAs of
+                // the previous item are done with it (this overlaps that item's
+                // epilogue, which reads O and M)
+                if (G > 0 && !mbar_wait(smem_u32(&bars->pv_done), (G - 1) & 1, wc)) break;
+                for (int c = 0; c < nchunk; ++c, ++kc) {
+                    const int s = kc % KST;
+                    if (!mbar_wait(smem_u32(&bars->k_full[s]), (kc / KST) & 1, wc)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_probe_chunk(sbase + Gm::OFF_K + s * Gm::K_BYTES, c == 0);
+                    tc_commit(smem_u32(&bars->k_empty[s]));
+                }
+                if (!ok) break;
+                tc_commit(smem_u32(&bars->r_tmem));
+            }
             for (int j = 0; j < it.nkv; ++j, ++G, ++kc) {
                 const int s = kc % KST;
                 if (!mbar_wait(smem_u32(&bars->k_full[s]), (kc / KST) & 1, wc)) { ok = false; break; }
@@ -401,6 +459,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 issue_scores(dq, kd);
                 tc_commit(smem_u32(&bars->s_full));
                 if constexpr (WITH_RHO) {
+                    // fused probe: the softmax warps have put R into shared memory
+                    if (FUSED && j == 0 && !mbar_wait(smem_u32(&bars->r_smem), ic & 1, wc)) { ok = false; break; }
                     if (!mbar_wait(smem_u32(&bars->s_free), G & 1, wc)) { ok = false; break; }
                     tc_fence_after();
                     issue_scores(dr, kd);
@@ -475,6 +535,37 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int qrow = it.qt * BM + r;
             const int kvis = causal ? min(T, qrow + 1) : T;  // keys visible to this row
             float m_ref = -INFINITY, l = 0.f, ab = 0.f;
+            if constexpr (FUSED) {
+                // ---- the probe tile R = X W_R of this item: TMEM (P region) ->
+                // bf16 -> shared memory, in the swizzled K-major layout a TMA
+                // load of rho would give, for the A UMMAs.  Group g converts
+                // columns [32g, 32g + 32) of its rows: the same TMEM columns it
+                // later overwrites with its P, so no group reads what another
+                // has already overwritten. ----
+                if (!warp_wait(smem_u32(&bars->r_tmem), ic & 1, wc)) { ok = false; break; }
+                tc_fence_after();
+                uint32_t rr[GCOLS];
+                tmem_ld16(tmem + lane_off + COL_P + grp * GCOLS, *reinterpret_cast<uint32_t(*)[16]>(&rr[0]));
+                tmem_ld16(tmem + lane_off + COL_P + grp * GCOLS + 16, *reinterpret_cast<uint32_t(*)[16]>(&rr[16]));
+                tmem_wait_ld();
+                uint8_t *rrow = smem + Gm::OFF_R + ((grp * GCOLS) / 64) * (Gm::Q_BYTES / Gm::HALVES) + r * 128;
+#pragma unroll
+                for (int c = 0; c < GCOLS / 8; ++c) {
+                    const int c16 = ((grp * GCOLS) % 64) / 8 + c;   // 16-byte chunk within the 128-byte row
+                    uint32_t pb[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(rr[8 * c + 2 * i]),
+                                                                       __uint_as_float(rr[8 * c + 2 * i + 1]));
+                        pb[i] = *reinterpret_cast<const uint32_t *>(&h);
+                    }
+                    *reinterpret_cast<uint4 *>(rrow + ((c16 ^ (r & 7)) << 4)) = make_uint4(pb[0], pb[1], pb[2], pb[3]);
+                }
+                fence_proxy_async_smem();   // read by the A UMMAs (async proxy)
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&bars->r_smem));
+            }
             for (int j = 0; j < it.nkv; ++j, ++G) {
                 // the exponent of this group's V block, needed only when P is stored
                 const int vblk = j * VPER + vsg;   // past the last block the keys read as zero
@@ -687,32 +778,45 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
 }
 
-template <int D, bool WITH_RHO, typename Tout>
-cudaError_t launch_t(const FwdTensorMaps &tm, void *y, float *lse, const signed char *vexp, int BH, int T,
-                     int causal, int sm_count, int *work_counter, const DeviceCtl &ctl, cudaStream_t s) {
+template <int D, bool WITH_RHO, bool FUSED, typename Tout>
+cudaError_t launch_t(const FwdTensorMaps &tm, void *y, float *lse, const signed char *vexp, int BH, int H, int T,
+                     int d_model, int causal, int sm_count, int *work_counter, const DeviceCtl &ctl, cudaStream_t s) {
     static std::atomic<unsigned long long> limit_set{0};
-    auto kern = k_fwd<D, WITH_RHO, Tout>;
+    auto kern = k_fwd<D, WITH_RHO, FUSED, Tout>;
     if (cudaError_t e = ensure_smem_limit(kern, (int)smem_bytes<D>(), limit_set)) return e;
     const int items = ((T + BM - 1) / BM) * BH;
     const int grid = items < sm_count ? items : sm_count;
     cudaError_t e = cudaMemsetAsync(work_counter, 0, sizeof(int), s);
     if (e != cudaSuccess) return e;
-    kern<<<grid, NTHREADS, smem_bytes<D>(), s>>>(tm.q, tm.k, tm.r, tm.v, static_cast<Tout *>(y), lse, vexp, BH, T,
-                                                 causal, work_counter, ctl);
+    kern<<<grid, NTHREADS, smem_bytes<D>(), s>>>(tm.q, tm.k, tm.r, tm.v, tm.x, tm.w, static_cast<Tout *>(y), lse,
+                                                 vexp, BH, H, T, d_model, causal, work_counter, ctl);
     return cudaGetLastError();
 }
 
-template <int D>
+template <int D, bool FUSED>
 cudaError_t launch_d(const FwdTensorMaps &tm, bool with_rho, void *y, float *lse, const signed char *vexp, int BH,
-                     int T, int causal, int out_dtype, int sm_count, int *work_counter, const DeviceCtl &ctl,
-                     cudaStream_t s) {
-    if (out_dtype == PARALLAX_F32) {
-        if (with_rho) return launch_t<D, true, float>(tm, y, lse, vexp, BH, T, causal, sm_count, work_counter, ctl, s);
-        return launch_t<D, false, float>(tm, y, lse, vexp, BH, T, causal, sm_count, work_counter, ctl, s);
+                     int H, int T, int d_model, int causal, int out_dtype, int sm_count, int *work_counter,
+                     const DeviceCtl &ctl, cudaStream_t s) {
+    if constexpr (FUSED) {
+        if (out_dtype == PARALLAX_F32)
+            return launch_t<D, true, true, float>(tm, y, lse, vexp, BH, H, T, d_model, causal, sm_count, work_counter,
+                                                  ctl, s);
+        return launch_t<D, true, true, __nv_bfloat16>(tm, y, lse, vexp, BH, H, T, d_model, causal, sm_count,
+                                                      work_counter, ctl, s);
+    } else {
+        if (out_dtype == PARALLAX_F32) {
+            if (with_rho)
+                return launch_t<D, true, false, float>(tm, y, lse, vexp, BH, H, T, 0, causal, sm_count, work_counter,
+                                                       ctl, s);
+            return launch_t<D, false, false, float>(tm, y, lse, vexp, BH, H, T, 0, causal, sm_count, work_counter,
+                                                    ctl, s);
+        }
+        if (with_rho)
+            return launch_t<D, true, false, __nv_bfloat16>(tm, y, lse, vexp, BH, H, T, 0, causal, sm_count,
+                                                           work_counter, ctl, s);
+        return launch_t<D, false, false, __nv_bfloat16>(tm, y, lse, vexp, BH, H, T, 0, causal, sm_count, work_counter,
+                                                        ctl, s);
     }
-    if (with_rho)
-        return launch_t<D, true, __nv_bfloat16>(tm, y, lse, vexp, BH, T, causal, sm_count, work_counter, ctl, s);
-    return launch_t<D, false, __nv_bfloat16>(tm, y, lse, vexp, BH, T, causal, sm_count, work_counter, ctl, s);
 }
 
 }  // namespace
@@ -721,8 +825,18 @@ cudaError_t launch_fwd_sm100(const FwdTensorMaps &tm, bool with_rho, void *y, fl
                              int B, int H, int T, int d, int causal, int out_dtype, int sm_count, int *work_counter,
                              const DeviceCtl &ctl, cudaStream_t s) {
     const int BH = B * H;
-    if (d == 64) return launch_d<64>(tm, with_rho, y, lse, vexp, BH, T, causal, out_dtype, sm_count, work_counter, ctl, s);
-    return launch_d<128>(tm, with_rho, y, lse, vexp, BH, T, causal, out_dtype, sm_count, work_counter, ctl, s);
+    if (d == 64)
+        return launch_d<64, false>(tm, with_rho, y, lse, vexp, BH, H, T, 0, causal, out_dtype, sm_count, work_counter,
+                                   ctl, s);
+    return launch_d<128, false>(tm, with_rho, y, lse, vexp, BH, H, T, 0, causal, out_dtype, sm_count, work_counter,
+                                ctl, s);
+}
+
+cudaError_t launch_fwd_fused_sm100(const FwdTensorMaps &tm, void *y, float *lse, const signed char *vexp, int B,
+                                   int H, int T, int d_model, int causal, int out_dtype, int sm_count,
+                                   int *work_counter, const DeviceCtl &ctl, cudaStream_t s) {
+    return launch_d<128, true>(tm, true, y, lse, vexp, B * H, H, T, d_model, causal, out_dtype, sm_count,
+                               work_counter, ctl, s);
 }
 
 }  // namespace plx

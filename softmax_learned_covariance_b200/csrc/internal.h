@@ -81,11 +81,17 @@ cudaError_t launch_v_to_f16_blocks(const void *v, void *v16, signed char *vexp, 
 // (tensor map `v` over the output of launch_v_to_f16_blocks, exponents in
 // `vexp`), fp32 accumulation, d in {64, 128}.  work_counter: one device int,
 // reset by the launch (stream-ordered), the persistent grid's item counter.
+// x, w: the fused probe's operands (x [B*T, d_model] and W_R [d_model, H*d],
+// 2-D, 128-byte swizzle, boxes 64 x 128 and 64 x 64); unused otherwise.
 struct FwdTensorMaps {
-    CUtensorMap q, k, r, v;
+    CUtensorMap q, k, r, v, x, w;
 };
 cudaError_t launch_fwd_sm100(const FwdTensorMaps &tm, bool with_rho, void *y, float *lse, const signed char *vexp,
                              int B, int H, int T, int d, int causal, int out_dtype, int sm_count, int *work_counter,
                              const DeviceCtl &ctl, cudaStream_t s);
+// The same forward with rho computed inside the kernel from x and W_R (d = 128).
+cudaError_t launch_fwd_fused_sm100(const FwdTensorMaps &tm, void *y, float *lse, const signed char *vexp, int B,
+                                   int H, int T, int d_model, int causal, int out_dtype, int sm_count,
+                                   int *work_counter, const DeviceCtl &ctl, cudaStream_t s);
 
 }  // namespace plx

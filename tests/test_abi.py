@@ -67,6 +67,18 @@ def test_fwd_host_validation(L):
     assert fwd(L, d=32, i=1, o=0) == 2      # head dims 64 and 128 only
 
 
+def test_fwd_fused_host_validation(L):
+    def ff(q=A16, k=A16, v=A16, x=A16, w=A16, y=A16, B=1, H=1, T=8, d=128, dm=128, i=1, o=0):
+        return L.parallax_fwd_fused(q, k, v, x, w, y, None, B, H, T, d, dm, 1, i, o, None)
+    assert ff(x=None) == 1
+    assert ff(w=None) == 1
+    assert ff(dm=100) == 2           # d_model must be a multiple of 64
+    assert ff(T=0) == 2
+    assert ff(w=MIS) == 3
+    assert ff(i=0) == 4              # bf16 inputs only
+    assert ff(d=64) == 5             # the fused probe is built for d = 128
+
+
 def test_decode_host_validation(L):
     def dec(q=A16, rho=A16, kc=A16, vc=A16, sl=A16, y=A16, B=2, H=2, Tcap=16, d=128, i=1, o=0):
         return L.parallax_decode(q, rho, kc, vc, sl, y, None, B, H, Tcap, d, i, o, None)
