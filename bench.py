@@ -472,6 +472,7 @@ def run_ours(args, rank, world):
         "decode_paged": extras["decode_paged"],
         "softmax_only_fwd": extras["softmax_only_fwd"],
         "fwd_fused": extras["fwd_fused"],
+        "bwd": extras["bwd"],
         "decode_long": decode_long,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
@@ -554,7 +555,27 @@ def measure_extras(args, stream, barrier, world, peaks, pc, dpq, dpk, dpv, yp, l
              "two_launch_ms": round(pipe_ms, 4), "speedup_vs_two_launch": round(pipe_ms / f_ms, 3),
              "note": "parallax_fwd_fused (rho computed per query tile in the kernel, never in HBM) vs "
                      "parallax_rho_proj + parallax_fwd on the same inputs; flops count both GEMM families"}
-    return {"decode_paged": paged, "softmax_only_fwd": smx, "fwd_fused": fused}
+    # ---- training: forward keeping o and abar, then the gradients ----
+    g = torch.Generator(device=dev)
+    g.manual_seed(13)
+    dpr = (torch.randn(dpq.shape, generator=g, device=dev) * 0.905).to(torch.bfloat16)
+    ddy = torch.randn(dpq.shape, generator=g, device=dev).to(torch.bfloat16)
+    with torch.cuda.stream(stream):
+        fwd_state = plx.parallax_fwd_train(dpq, dpk, dpv, dpr, stream=stream)
+        tr_ms = timed(lambda: plx.parallax_fwd_train(dpq, dpk, dpv, dpr, stream=stream), max(2, args.steps // 4))
+        b_ms = timed(lambda: plx.parallax_bwd(dpq, dpk, dpv, dpr, *fwd_state[:1], fwd_state[2], fwd_state[3],
+                                              fwd_state[1], ddy, stream=stream), max(2, args.steps // 4))
+    assert plx.parallax_last_device_error(stream) == 0
+    b_flops = 16 * pc["d"] * pairs   # dV, dK (two), dQ, dR and the three recomputed score products: 8 GEMMs
+    bwd = {"ms": round(b_ms, 4), "tflops": round(b_flops / (b_ms * 1e-3) / 1e12, 2), "flops": b_flops,
+           "roofline": {"bound": "tensor", "achieved": round(b_flops / (b_ms * 1e-3) / 1e12, 2),
+                        "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                        "frac": round(b_flops / (b_ms * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)},
+           "fwd_train_ms": round(tr_ms, 4),
+           "note": "parallax_bwd (mma.sync kernels; scores recomputed in both, 11 products executed per pair) "
+                   "after parallax_fwd_train on the prefill shape; flops count 8 GEMMs of 2d per pair"}
+    del dpr, ddy, fwd_state
+    return {"decode_paged": paged, "softmax_only_fwd": smx, "fwd_fused": fused, "bwd": bwd}
 
 
 # --------------------------------------------------------------------------- #

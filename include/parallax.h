@@ -136,6 +136,41 @@ PARALLAX_API int parallax_fwd_fused(const void *q, const void *k, const void *v,
                                     int in_dtype, int out_dtype, parallax_stream_t stream);
 
 /*
+ * parallax_fwd_train -- parallax_fwd that also keeps what the backward needs.
+ *
+ * Same operator and tensor-core kernel as parallax_fwd (bf16 inputs, fp32 y),
+ * and also writes, per row, the softmax attention output o_i = sum_j s_ij v_j
+ * and abar_i = sum_j s_ij a_ij.
+ *   q, k, v, rho : [B, H, T, d] bf16 (rho required).
+ *   y, o         : [B, H, T, d] fp32 (written);  lse, abar : [B, H, T] fp32 (written).
+ *   d in {64, 128}; in_dtype must be BF16.  Scratch as parallax_fwd.
+ */
+PARALLAX_API int parallax_fwd_train(const void *q, const void *k, const void *v, const void *rho, float *y,
+                                    float *lse, float *o, float *abar, int B, int H, int T, int d, int causal,
+                                    int in_dtype, parallax_stream_t stream);
+
+/*
+ * parallax_bwd -- gradients of the prefill with respect to q, k, v and rho.
+ *
+ * The pages train with this operator (encorp.ai blog, section "Las ganancias
+ * de preentrenamiento..."; zubnet.ai news item on Parallax, paragraph 1); the
+ * gradients are the chain rule through the definitions above, for a loss L
+ * with dL/dy = dy.  Chain to W_R through rho = x W_R with the caller's GEMMs.
+ *   q, k, v, rho, dy : [B, H, T, d] bf16.
+ *   y, o, abar, lse  : the outputs of parallax_fwd_train on the same inputs.
+ *   dq, dk, dv, drho : [B, H, T, d] fp32 (written, not accumulated).
+ *   d in {64, 128}; B * H <= 65535; in_dtype must be BF16.
+ * Warp-level tensor-core kernels (mma.sync): one over query blocks for dq and
+ * drho, one over key blocks for dk and dv, both recomputing the scores, so no
+ * gradient is accumulated with atomics and the result is deterministic.
+ * Scratch: 8 bytes per row (see the conventions above).
+ */
+PARALLAX_API int parallax_bwd(const void *q, const void *k, const void *v, const void *rho, const float *y,
+                              const float *o, const float *abar, const float *lse, const void *dy, float *dq,
+                              float *dk, float *dv, float *drho, int B, int H, int T, int d, int causal,
+                              int in_dtype, parallax_stream_t stream);
+
+/*
  * parallax_decode -- one new query token per sequence against a KV cache.
  *
  * Passage: zubnet.ai news item on Parallax, paragraph 2 (the KV cache is still

@@ -12,6 +12,8 @@ library is missing or a call fails, a ``ParallaxError`` is raised.
 Functions keep the C names:
     parallax_fwd(q, k, v, rho=None, causal=True, out_dtype=torch.float32) -> (y, lse)
     parallax_fwd_fused(q, k, v, x, W_R, causal=True) -> (y, lse)     probe rho = x W_R in the kernel
+    parallax_fwd_train(q, k, v, rho, causal=True) -> (y, lse, o, abar)  the forward kept for the backward
+    parallax_bwd(q, k, v, rho, y, o, abar, lse, dy, causal=True) -> (dq, dk, dv, drho)
     parallax_decode(q, rho, kcache, vcache, seqlens, out_dtype=torch.float32) -> (y, lse)
     parallax_decode_ex(..., workspace) -> (y, lse)          caller-owned split scratch
     parallax_decode_paged(q, rho, kpages, vpages, block_table, seqlens) -> (y, lse)
@@ -25,7 +27,8 @@ import os
 import threading
 
 __all__ = [
-    "ParallaxError", "lib", "parallax_fwd", "parallax_fwd_fused", "parallax_decode", "parallax_decode_ex", "parallax_decode_paged",
+    "ParallaxError", "lib", "parallax_fwd", "parallax_fwd_fused", "parallax_fwd_train", "parallax_bwd",
+    "parallax_decode", "parallax_decode_ex", "parallax_decode_paged",
     "parallax_rho_proj", "parallax_decode_workspace_bytes", "parallax_last_device_error",
     "parallax_strerror", "parallax_device_sm_count", "LIB_PATH", "F32", "BF16",
 ]
@@ -54,6 +57,8 @@ def lib() -> ctypes.CDLL:
             P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
             L.parallax_fwd.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, P]
             L.parallax_fwd_fused.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P]
+            L.parallax_fwd_train.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, P]
+            L.parallax_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, P]
             L.parallax_decode.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, P]
             L.parallax_decode_ex.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, P, S, P]
             L.parallax_decode_paged.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, P]
@@ -64,7 +69,7 @@ def lib() -> ctypes.CDLL:
             L.parallax_strerror.restype = ctypes.c_char_p
             L.parallax_last_device_error.argtypes = [P]
             L.parallax_device_sm_count.argtypes = []
-            for f in (L.parallax_fwd, L.parallax_fwd_fused, L.parallax_decode, L.parallax_decode_ex, L.parallax_decode_paged,
+            for f in (L.parallax_fwd, L.parallax_fwd_fused, L.parallax_fwd_train, L.parallax_bwd, L.parallax_decode, L.parallax_decode_ex, L.parallax_decode_paged,
                       L.parallax_rho_proj,
                       L.parallax_last_device_error, L.parallax_device_sm_count):
                 f.restype = I
@@ -159,6 +164,36 @@ def parallax_fwd_fused(q, k, v, x, W_R, causal: bool = True, out_dtype=None, y=N
                                   _stream(stream))
     _check(st, "parallax_fwd_fused")
     return y, lse
+
+
+def parallax_fwd_train(q, k, v, rho, causal: bool = True, stream=None):
+    """Training forward: (y, lse, o, abar), fp32; o and abar are what parallax_bwd needs."""
+    torch = _torch()
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (rho, "rho")):
+        _need(t, n)
+    B, H, T, d = q.shape
+    f32 = dict(dtype=torch.float32, device=q.device)
+    y, o = torch.empty((B, H, T, d), **f32), torch.empty((B, H, T, d), **f32)
+    lse, abar = torch.empty((B, H, T), **f32), torch.empty((B, H, T), **f32)
+    st = lib().parallax_fwd_train(_ptr(q), _ptr(k), _ptr(v), _ptr(rho), _ptr(y), _ptr(lse), _ptr(o), _ptr(abar),
+                                  B, H, T, d, int(bool(causal)), _dtype_code(q.dtype), _stream(stream))
+    _check(st, "parallax_fwd_train")
+    return y, lse, o, abar
+
+
+def parallax_bwd(q, k, v, rho, y, o, abar, lse, dy, causal: bool = True, stream=None):
+    """Gradients (dq, dk, dv, drho), fp32, for an upstream dy (bf16, [B, H, T, d])."""
+    torch = _torch()
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (rho, "rho"), (y, "y"), (o, "o"), (abar, "abar"), (lse, "lse"),
+                 (dy, "dy")):
+        _need(t, n)
+    B, H, T, d = q.shape
+    outs = [torch.empty((B, H, T, d), dtype=torch.float32, device=q.device) for _ in range(4)]
+    st = lib().parallax_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(rho), _ptr(y), _ptr(o), _ptr(abar), _ptr(lse), _ptr(dy),
+                            *(_ptr(t) for t in outs), B, H, T, d, int(bool(causal)), _dtype_code(q.dtype),
+                            _stream(stream))
+    _check(st, "parallax_bwd")
+    return tuple(outs)
 
 
 def parallax_decode(q, rho, kcache, vcache, seqlens, out_dtype=None, y=None, lse=None, stream=None,

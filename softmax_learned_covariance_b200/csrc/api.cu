@@ -251,9 +251,59 @@ int parallax_fwd(const void *q, const void *k, const void *v, const void *rho, v
         const uint32_t box_q[3] = {64, 128, 1};
         if ((st = encode(&tm.r, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rho, 3, dims, box_q, 2))) return st;
     }
-    return status_of(
-        launch_fwd_sm100(tm, rho != nullptr, y, lse, vexp, B, H, T, d, causal, out_dtype, s->sms, counter, make_ctl(s),
-                         cs));
+    return status_of(launch_fwd_sm100(tm, rho != nullptr, y, lse, nullptr, nullptr, vexp, B, H, T, d, causal,
+                                      out_dtype, s->sms, counter, make_ctl(s), cs));
+}
+
+int parallax_fwd_train(const void *q, const void *k, const void *v, const void *rho, float *y, float *lse, float *o,
+                       float *abar, int B, int H, int T, int d, int causal, int in_dtype, parallax_stream_t stream) {
+    if (!q || !k || !v || !rho || !y || !lse || !o || !abar) return PARALLAX_ERR_NULL;
+    if (B < 1 || H < 1 || T < 1 || (d != 64 && d != 128)) return PARALLAX_ERR_SHAPE;
+    if ((long long)B * H * T * d > (1ll << 40) || (long long)B * H > (1ll << 30)) return PARALLAX_ERR_SHAPE;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(rho) || !aligned16(y) || !aligned16(o) ||
+        !aligned4(lse) || !aligned4(abar))
+        return PARALLAX_ERR_ALIGN;
+    if (in_dtype != PARALLAX_BF16) return PARALLAX_ERR_DTYPE;
+    DevState *s = nullptr;
+    int st = get_state(&s);
+    if (st) return st;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if ((st = ensure_encoder())) return st;
+    CallScratch scratch(s, cs);
+    FwdTensorMaps tm;
+    signed char *vexp = nullptr;
+    int *counter = nullptr;
+    if ((st = prepare_fwd(q, k, v, B, H, T, d, cs, scratch, &tm, &vexp, &counter))) return st;
+    const uint64_t dims[3] = {(uint64_t)d, (uint64_t)T, (uint64_t)B * H};
+    const uint32_t box_q[3] = {64, 128, 1};
+    if ((st = encode(&tm.r, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rho, 3, dims, box_q, 2))) return st;
+    return status_of(launch_fwd_sm100(tm, true, y, lse, o, abar, vexp, B, H, T, d, causal, PARALLAX_F32, s->sms,
+                                      counter, make_ctl(s), cs));
+}
+
+int parallax_bwd(const void *q, const void *k, const void *v, const void *rho, const float *y, const float *o,
+                 const float *abar, const float *lse, const void *dy, float *dq, float *dk, float *dv, float *drho,
+                 int B, int H, int T, int d, int causal, int in_dtype, parallax_stream_t stream) {
+    if (!q || !k || !v || !rho || !y || !o || !abar || !lse || !dy || !dq || !dk || !dv || !drho)
+        return PARALLAX_ERR_NULL;
+    if (B < 1 || H < 1 || T < 1 || (d != 64 && d != 128)) return PARALLAX_ERR_SHAPE;
+    if ((long long)B * H * T * d > (1ll << 40) || (long long)B * H > 65535) return PARALLAX_ERR_SHAPE;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(rho) || !aligned16(y) || !aligned16(o) ||
+        !aligned16(dy) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(drho) || !aligned4(abar) ||
+        !aligned4(lse))
+        return PARALLAX_ERR_ALIGN;
+    if (in_dtype != PARALLAX_BF16) return PARALLAX_ERR_DTYPE;
+    DevState *s = nullptr;
+    int st = get_state(&s);
+    if (st) return st;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    // scratch: go and delta per row
+    CallScratch scratch(s, cs);
+    void *ws = nullptr;
+    const size_t rows = (size_t)B * H * T;
+    if ((st = scratch.get(2 * rows * sizeof(float), &ws))) return st;
+    float *go = static_cast<float *>(ws), *delta = go + rows;
+    return status_of(launch_bwd(q, k, v, rho, dy, y, o, abar, lse, go, delta, dq, dk, dv, drho, B, H, T, d, causal, cs));
 }
 
 int parallax_fwd_fused(const void *q, const void *k, const void *v, const void *x, const void *W_R, void *y,

@@ -229,8 +229,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     k_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
           const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_v,
           const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w, Tout *__restrict__ y,
-          float *__restrict__ lse, const signed char *__restrict__ vexp_g, int BH, int H, int T, int d_model,
-          int causal, int *__restrict__ work_counter, DeviceCtl ctl) {
+          float *__restrict__ lse, float *__restrict__ o_out, float *__restrict__ abar_out,
+          const signed char *__restrict__ vexp_g, int BH, int H, int T, int d_model, int causal,
+          int *__restrict__ work_counter, DeviceCtl ctl) {
     using Gm = Geo<D>;
     static_assert(!FUSED || (WITH_RHO && D == 128), "the fused probe needs the correction branch and d = 128");
     // fused probe: X W_R is accumulated over d_model in chunks of 64 that
@@ -743,6 +744,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     }
                     finite = finite && isfinite(out[i]);
                 }
+                if (store && o_out != nullptr) {   // training forward: o = O / l for the backward
+                    float4 *dst = reinterpret_cast<float4 *>(o_out + ((size_t)it.bh * T + qrow) * D + c);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv_l, __uint_as_float(o[4 * i + 1]) * inv_l,
+                                             __uint_as_float(o[4 * i + 2]) * inv_l,
+                                             __uint_as_float(o[4 * i + 3]) * inv_l);
+                }
                 if (store) {
                     if constexpr (sizeof(Tout) == 4) {
                         float4 *dst = reinterpret_cast<float4 *>(yrow + c);
@@ -763,6 +772,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
             }
             if (store && grp == 0 && lse != nullptr) lse[(size_t)it.bh * T + qrow] = (m_ref + log2f(lt)) * LN2;
+            if (store && grp == 0 && abar_out != nullptr) abar_out[(size_t)it.bh * T + qrow] = abar * A_UNSCALE;
             // an output that is not finite: an input outside the kernel's range
             if (__any_sync(0xffffffffu, store && !finite) && lane == 0) atomicCAS(ctl.err, 0, PARALLAX_ERR_DEVICE_RANGE);
             tc_fence_before();
@@ -779,8 +789,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 }
 
 template <int D, bool WITH_RHO, bool FUSED, typename Tout>
-cudaError_t launch_t(const FwdTensorMaps &tm, void *y, float *lse, const signed char *vexp, int BH, int H, int T,
-                     int d_model, int causal, int sm_count, int *work_counter, const DeviceCtl &ctl, cudaStream_t s) {
+cudaError_t launch_t(const FwdTensorMaps &tm, void *y, float *lse, float *o_out, float *abar_out,
+                     const signed char *vexp, int BH, int H, int T, int d_model, int causal, int sm_count,
+                     int *work_counter, const DeviceCtl &ctl, cudaStream_t s) {
     static std::atomic<unsigned long long> limit_set{0};
     auto kern = k_fwd<D, WITH_RHO, FUSED, Tout>;
     if (cudaError_t e = ensure_smem_limit(kern, (int)smem_bytes<D>(), limit_set)) return e;
@@ -789,54 +800,54 @@ cudaError_t launch_t(const FwdTensorMaps &tm, void *y, float *lse, const signed 
     cudaError_t e = cudaMemsetAsync(work_counter, 0, sizeof(int), s);
     if (e != cudaSuccess) return e;
     kern<<<grid, NTHREADS, smem_bytes<D>(), s>>>(tm.q, tm.k, tm.r, tm.v, tm.x, tm.w, static_cast<Tout *>(y), lse,
-                                                 vexp, BH, H, T, d_model, causal, work_counter, ctl);
+                                                 o_out, abar_out, vexp, BH, H, T, d_model, causal, work_counter, ctl);
     return cudaGetLastError();
 }
 
 template <int D, bool FUSED>
-cudaError_t launch_d(const FwdTensorMaps &tm, bool with_rho, void *y, float *lse, const signed char *vexp, int BH,
-                     int H, int T, int d_model, int causal, int out_dtype, int sm_count, int *work_counter,
-                     const DeviceCtl &ctl, cudaStream_t s) {
+cudaError_t launch_d(const FwdTensorMaps &tm, bool with_rho, void *y, float *lse, float *o_out, float *abar_out,
+                     const signed char *vexp, int BH, int H, int T, int d_model, int causal, int out_dtype,
+                     int sm_count, int *work_counter, const DeviceCtl &ctl, cudaStream_t s) {
     if constexpr (FUSED) {
         if (out_dtype == PARALLAX_F32)
-            return launch_t<D, true, true, float>(tm, y, lse, vexp, BH, H, T, d_model, causal, sm_count, work_counter,
+            return launch_t<D, true, true, float>(tm, y, lse, o_out, abar_out, vexp, BH, H, T, d_model, causal, sm_count, work_counter,
                                                   ctl, s);
-        return launch_t<D, true, true, __nv_bfloat16>(tm, y, lse, vexp, BH, H, T, d_model, causal, sm_count,
+        return launch_t<D, true, true, __nv_bfloat16>(tm, y, lse, o_out, abar_out, vexp, BH, H, T, d_model, causal, sm_count,
                                                       work_counter, ctl, s);
     } else {
         if (out_dtype == PARALLAX_F32) {
             if (with_rho)
-                return launch_t<D, true, false, float>(tm, y, lse, vexp, BH, H, T, 0, causal, sm_count, work_counter,
+                return launch_t<D, true, false, float>(tm, y, lse, o_out, abar_out, vexp, BH, H, T, 0, causal, sm_count, work_counter,
                                                        ctl, s);
-            return launch_t<D, false, false, float>(tm, y, lse, vexp, BH, H, T, 0, causal, sm_count, work_counter,
+            return launch_t<D, false, false, float>(tm, y, lse, o_out, abar_out, vexp, BH, H, T, 0, causal, sm_count, work_counter,
                                                     ctl, s);
         }
         if (with_rho)
-            return launch_t<D, true, false, __nv_bfloat16>(tm, y, lse, vexp, BH, H, T, 0, causal, sm_count,
+            return launch_t<D, true, false, __nv_bfloat16>(tm, y, lse, o_out, abar_out, vexp, BH, H, T, 0, causal, sm_count,
                                                            work_counter, ctl, s);
-        return launch_t<D, false, false, __nv_bfloat16>(tm, y, lse, vexp, BH, H, T, 0, causal, sm_count, work_counter,
+        return launch_t<D, false, false, __nv_bfloat16>(tm, y, lse, o_out, abar_out, vexp, BH, H, T, 0, causal, sm_count, work_counter,
                                                         ctl, s);
     }
 }
 
 }  // namespace
 
-cudaError_t launch_fwd_sm100(const FwdTensorMaps &tm, bool with_rho, void *y, float *lse, const signed char *vexp,
-                             int B, int H, int T, int d, int causal, int out_dtype, int sm_count, int *work_counter,
-                             const DeviceCtl &ctl, cudaStream_t s) {
+cudaError_t launch_fwd_sm100(const FwdTensorMaps &tm, bool with_rho, void *y, float *lse, float *o_out,
+                             float *abar_out, const signed char *vexp, int B, int H, int T, int d, int causal,
+                             int out_dtype, int sm_count, int *work_counter, const DeviceCtl &ctl, cudaStream_t s) {
     const int BH = B * H;
     if (d == 64)
-        return launch_d<64, false>(tm, with_rho, y, lse, vexp, BH, H, T, 0, causal, out_dtype, sm_count, work_counter,
-                                   ctl, s);
-    return launch_d<128, false>(tm, with_rho, y, lse, vexp, BH, H, T, 0, causal, out_dtype, sm_count, work_counter,
-                                ctl, s);
+        return launch_d<64, false>(tm, with_rho, y, lse, o_out, abar_out, vexp, BH, H, T, 0, causal, out_dtype,
+                                   sm_count, work_counter, ctl, s);
+    return launch_d<128, false>(tm, with_rho, y, lse, o_out, abar_out, vexp, BH, H, T, 0, causal, out_dtype, sm_count,
+                                work_counter, ctl, s);
 }
 
 cudaError_t launch_fwd_fused_sm100(const FwdTensorMaps &tm, void *y, float *lse, const signed char *vexp, int B,
                                    int H, int T, int d_model, int causal, int out_dtype, int sm_count,
                                    int *work_counter, const DeviceCtl &ctl, cudaStream_t s) {
-    return launch_d<128, true>(tm, true, y, lse, vexp, B * H, H, T, d_model, causal, out_dtype, sm_count,
-                               work_counter, ctl, s);
+    return launch_d<128, true>(tm, true, y, lse, nullptr, nullptr, vexp, B * H, H, T, d_model, causal, out_dtype,
+                               sm_count, work_counter, ctl, s);
 }
 
 }  // namespace plx

@@ -86,12 +86,21 @@ cudaError_t launch_v_to_f16_blocks(const void *v, void *v16, signed char *vexp, 
 struct FwdTensorMaps {
     CUtensorMap q, k, r, v, x, w;
 };
-cudaError_t launch_fwd_sm100(const FwdTensorMaps &tm, bool with_rho, void *y, float *lse, const signed char *vexp,
-                             int B, int H, int T, int d, int causal, int out_dtype, int sm_count, int *work_counter,
-                             const DeviceCtl &ctl, cudaStream_t s);
+// o_out [B,H,T,d] fp32 and abar_out [B,H,T] fp32 (nullable): the softmax
+// attention output o and abar of each row, kept for the backward.
+cudaError_t launch_fwd_sm100(const FwdTensorMaps &tm, bool with_rho, void *y, float *lse, float *o_out,
+                             float *abar_out, const signed char *vexp, int B, int H, int T, int d, int causal,
+                             int out_dtype, int sm_count, int *work_counter, const DeviceCtl &ctl, cudaStream_t s);
 // The same forward with rho computed inside the kernel from x and W_R (d = 128).
 cudaError_t launch_fwd_fused_sm100(const FwdTensorMaps &tm, void *y, float *lse, const signed char *vexp, int B,
                                    int H, int T, int d_model, int causal, int out_dtype, int sm_count,
                                    int *work_counter, const DeviceCtl &ctl, cudaStream_t s);
+
+// Gradients of the prefill (mma.sync kernels): go, delta are [B*H*T] fp32
+// scratch; q, k, v, rho, dy bf16; y, o fp32 [B,H,T,d]; abar, lse fp32 [B,H,T];
+// dq, dk, dv, drho fp32 [B,H,T,d] (written).
+cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *rho, const void *dy, const float *y,
+                       const float *o, const float *abar, const float *lse, float *go, float *delta, float *dq,
+                       float *dk, float *dv, float *drho, int B, int H, int T, int d, int causal, cudaStream_t s);
 
 }  // namespace plx
