@@ -166,6 +166,7 @@ def run_profile_case(args):
     profile_decode : parallax_decode, B=16 H=16 d=128, 8192-token cache
     profile_rho    : parallax_rho_proj, x [2, 8192, 2048] @ W_R [2048, 2048]
     profile_paged  : parallax_decode_paged, B=64 Hq=32 Hkv=8, 64-token pages, ctx 4096 (1.07 GB)
+    profile_bwd    : parallax_bwd, B=2 H=16 T=4096 d=128 causal (after one parallax_fwd_train)
     """
     import torch
 
@@ -205,6 +206,14 @@ def run_profile_case(args):
         call = lambda: plx.parallax_decode_paged(q, r, kp, vp, tb, dsl, y=y, want_lse=False)
         work = c["B"] * c["Hkv"] * c["ctx"] * c["d"] * 4 + c["B"] * c["Hq"] * c["d"] * 8
         unit = "TB/s"
+    elif args.workload == "profile_bwd":
+        g = torch.Generator(device=dev)
+        g.manual_seed(1)
+        mk = lambda s=1.0: (torch.randn((2, 16, 4096, 128), generator=g, device=dev) * s).to(torch.bfloat16)
+        q, k, v, r, dy = mk(), mk(), mk(), mk(0.905), mk()
+        y, lse, o, abar = plx.parallax_fwd_train(q, k, v, r)
+        call = lambda: plx.parallax_bwd(q, k, v, r, y, o, abar, lse, dy)
+        work, unit = 16 * 128 * prefill_pairs(2, 16, 4096), "TFLOP/s"
     else:
         x, w = (t.torch().to(dev) for t in inputs.rho_proj_inputs(2, 8192, 2048, 16, 128, seed=3))
         r = torch.empty((2, 16, 8192, 128), dtype=torch.bfloat16, device=dev)
@@ -473,6 +482,9 @@ def run_ours(args, rank, world):
         "softmax_only_fwd": extras["softmax_only_fwd"],
         "fwd_fused": extras["fwd_fused"],
         "bwd": extras["bwd"],
+        "softmax_decode": dict(extras["softmax_decode"],
+                               parallax_over_io_matched=round(dec_ms / extras["softmax_decode"]["d"]["ms"], 3),
+                               parallax_over_compute_matched=round(dec_ms / extras["softmax_decode"]["2d"]["ms"], 3)),
         "decode_long": decode_long,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
@@ -546,6 +558,31 @@ def measure_extras(args, stream, barrier, world, peaks, pc, dpq, dpk, dpv, yp, l
     smx = {"ms": round(s_ms, 4), "tflops": round(s_tf, 2), "flops": 4 * pc["d"] * pairs,
            "parallax_over_softmax_time": round(fwd_ms / s_ms, 3),
            "note": "rho = NULL instantiation of the same kernel (2 of the 4 GEMMs); same inputs and shape"}
+    # ---- softmax attention decode, the pages' comparison baseline: at the same
+    # head dim (same KV bytes: I/O-matched) and at twice it (same arithmetic per
+    # cached token: compute-matched), on the decode step's shape ----
+    dc = DECODE_CFG
+    gsd = torch.Generator(device=dev)
+    gsd.manual_seed(17)
+    sd = {}
+    for dd in (dc["d"], 2 * dc["d"]):
+        qs = torch.randn((dc["B"], dc["H"], dd), generator=gsd, device=dev).to(torch.bfloat16)
+        kcs = torch.randn((dc["B"], dc["H"], dc["Tcap"], dd), generator=gsd, device=dev).to(torch.bfloat16)
+        vcs = torch.randn((dc["B"], dc["H"], dc["Tcap"], dd), generator=gsd, device=dev).to(torch.bfloat16)
+        sls = torch.full((dc["B"],), dc["Tcap"], dtype=torch.int32, device=dev)
+        ys = torch.empty((dc["B"], dc["H"], dd), dtype=torch.float32, device=dev)
+        with torch.cuda.stream(stream):
+            ms_ = timed(lambda: plx.parallax_softmax_decode(qs, kcs, vcs, sls, y=ys, want_lse=False, stream=stream),
+                        args.steps)
+        nb = decode_bytes(dc["B"], dc["H"], dd, np.full((dc["B"],), dc["Tcap"])) - dc["B"] * dc["H"] * dd * 2
+        sd[dd] = {"ms": round(ms_, 4), "GB/s": round(nb / (ms_ * 1e-3) / 1e9, 1)}
+        del qs, kcs, vcs, sls, ys
+    torch.cuda.empty_cache()
+    softmax_decode = {"d": sd[dc["d"]], "2d": sd[2 * dc["d"]],
+                      "note": "parallax_softmax_decode on B=64 H=16 ctx 4096; ratios are the Parallax decode "
+                              "call's time over these (> 1 means Parallax is slower)",
+                      "parallax_over_io_matched": None, "parallax_over_compute_matched": None}
+
     # ---- probe rho = x W_R inside the prefill kernel ----
     with torch.cuda.stream(stream):
         f_ms = timed(lambda: plx.parallax_fwd_fused(dpq, dpk, dpv, dx, dw, y=yp, lse=lp, stream=stream), args.steps)
@@ -575,7 +612,8 @@ def measure_extras(args, stream, barrier, world, peaks, pc, dpq, dpk, dpv, yp, l
            "note": "parallax_bwd (mma.sync kernels; scores recomputed in both, 11 products executed per pair) "
                    "after parallax_fwd_train on the prefill shape; flops count 8 GEMMs of 2d per pair"}
     del dpr, ddy, fwd_state
-    return {"decode_paged": paged, "softmax_only_fwd": smx, "fwd_fused": fused, "bwd": bwd}
+    return {"decode_paged": paged, "softmax_only_fwd": smx, "fwd_fused": fused, "bwd": bwd,
+            "softmax_decode": softmax_decode}
 
 
 # --------------------------------------------------------------------------- #
@@ -648,7 +686,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["default", "prefill_long", "sweep", "profile_fwd", "profile_decode",
-                                           "profile_rho", "profile_paged", "profile_fwd_long"], default="default")
+                                           "profile_rho", "profile_paged", "profile_fwd_long", "profile_bwd"],
+                    default="default")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode-long", action="store_true", help="skip the long-context decode cells")

@@ -193,6 +193,24 @@ PARALLAX_API int parallax_decode(const void *q, const void *rho, const void *kca
                     const int *seqlens, void *y, float *lse, int B, int H, int Tcap, int d,
                     int in_dtype, int out_dtype, parallax_stream_t stream);
 
+/*
+ * parallax_softmax_decode -- plain softmax attention decode, the reference the
+ * pages compare the Parallax decode with.
+ *
+ * Passage: encorp.ai blog, section "Como cambia Parallax la historia del
+ * hardware en GPU Hopper", and zubnet.ai news item on Parallax, paragraph 2
+ * (decode against FlashAttention 2/3, "compute-matched" and "I/O-matched").
+ * The same split kernel as parallax_decode with the probe branch removed:
+ * y = sum_j s_j v_j.  Head dims 64, 128 and 256: at the same d it reads the
+ * same KV bytes as parallax_decode (I/O-matched); at 2d it does the same
+ * arithmetic per cached token (compute-matched).
+ *   q : [B, H, d] bf16;  kcache, vcache : [B, H, Tcap, d] bf16;
+ *   seqlens, y, lse, dtypes and scratch as parallax_decode.
+ */
+PARALLAX_API int parallax_softmax_decode(const void *q, const void *kcache, const void *vcache, const int *seqlens,
+                                         void *y, float *lse, int B, int H, int Tcap, int d, int in_dtype,
+                                         int out_dtype, parallax_stream_t stream);
+
 /* Bytes of scratch parallax_decode_ex needs for this shape on the current
  * device (0 if it needs none, or on a bad shape or CUDA error). */
 PARALLAX_API size_t parallax_decode_workspace_bytes(int B, int H, int Tcap, int d);

@@ -15,6 +15,7 @@ Functions keep the C names:
     parallax_fwd_train(q, k, v, rho, causal=True) -> (y, lse, o, abar)  the forward kept for the backward
     parallax_bwd(q, k, v, rho, y, o, abar, lse, dy, causal=True) -> (dq, dk, dv, drho)
     parallax_decode(q, rho, kcache, vcache, seqlens, out_dtype=torch.float32) -> (y, lse)
+    parallax_softmax_decode(q, kcache, vcache, seqlens) -> (y, lse)   reference: softmax attention, d 64/128/256
     parallax_decode_ex(..., workspace) -> (y, lse)          caller-owned split scratch
     parallax_decode_paged(q, rho, kpages, vpages, block_table, seqlens) -> (y, lse)
                                                             paged cache, grouped query heads
@@ -28,7 +29,7 @@ import threading
 
 __all__ = [
     "ParallaxError", "lib", "parallax_fwd", "parallax_fwd_fused", "parallax_fwd_train", "parallax_bwd",
-    "parallax_decode", "parallax_decode_ex", "parallax_decode_paged",
+    "parallax_decode", "parallax_softmax_decode", "parallax_decode_ex", "parallax_decode_paged",
     "parallax_rho_proj", "parallax_decode_workspace_bytes", "parallax_last_device_error",
     "parallax_strerror", "parallax_device_sm_count", "LIB_PATH", "F32", "BF16",
 ]
@@ -60,6 +61,7 @@ def lib() -> ctypes.CDLL:
             L.parallax_fwd_train.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, P]
             L.parallax_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, P]
             L.parallax_decode.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, P]
+            L.parallax_softmax_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P]
             L.parallax_decode_ex.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, P, S, P]
             L.parallax_decode_paged.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, P]
             L.parallax_decode_workspace_bytes.argtypes = [I, I, I, I]
@@ -69,7 +71,8 @@ def lib() -> ctypes.CDLL:
             L.parallax_strerror.restype = ctypes.c_char_p
             L.parallax_last_device_error.argtypes = [P]
             L.parallax_device_sm_count.argtypes = []
-            for f in (L.parallax_fwd, L.parallax_fwd_fused, L.parallax_fwd_train, L.parallax_bwd, L.parallax_decode, L.parallax_decode_ex, L.parallax_decode_paged,
+            for f in (L.parallax_fwd, L.parallax_fwd_fused, L.parallax_fwd_train, L.parallax_bwd, L.parallax_decode,
+                      L.parallax_softmax_decode, L.parallax_decode_ex, L.parallax_decode_paged,
                       L.parallax_rho_proj,
                       L.parallax_last_device_error, L.parallax_device_sm_count):
                 f.restype = I
@@ -214,6 +217,24 @@ def parallax_decode(q, rho, kcache, vcache, seqlens, out_dtype=None, y=None, lse
                                _ptr(lse), B, H, Tcap, d, _dtype_code(q.dtype), _dtype_code(y.dtype),
                                _stream(stream))
     _check(st, "parallax_decode")
+    return y, lse
+
+
+def parallax_softmax_decode(q, kcache, vcache, seqlens, out_dtype=None, y=None, lse=None, stream=None,
+                            want_lse: bool = True):
+    """Plain softmax attention decode (no probe), head dims 64, 128, 256: the pages' reference point."""
+    torch = _torch()
+    for t, n in ((q, "q"), (kcache, "kcache"), (vcache, "vcache"), (seqlens, "seqlens")):
+        _need(t, n)
+    B, H, Tcap, d = kcache.shape
+    out_dtype = out_dtype or torch.float32
+    if y is None:
+        y = torch.empty((B, H, d), dtype=out_dtype, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    st = lib().parallax_softmax_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens), _ptr(y), _ptr(lse), B, H,
+                                       Tcap, d, _dtype_code(q.dtype), _dtype_code(y.dtype), _stream(stream))
+    _check(st, "parallax_softmax_decode")
     return y, lse
 
 

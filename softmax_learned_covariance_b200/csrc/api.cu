@@ -386,6 +386,28 @@ int parallax_decode(const void *q, const void *rho, const void *kcache, const vo
                        stream);
 }
 
+int parallax_softmax_decode(const void *q, const void *kcache, const void *vcache, const int *seqlens, void *y,
+                            float *lse, int B, int H, int Tcap, int d, int in_dtype, int out_dtype,
+                            parallax_stream_t stream) {
+    if (!q || !kcache || !vcache || !seqlens || !y) return PARALLAX_ERR_NULL;
+    if (B < 1 || H < 1 || Tcap < 1 || (d != 64 && d != 128 && d != 256)) return PARALLAX_ERR_SHAPE;
+    if ((long long)B * H * Tcap * d > (1ll << 40)) return PARALLAX_ERR_SHAPE;
+    if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned4(seqlens) || !aligned16(y) ||
+        (lse && !aligned4(lse)))
+        return PARALLAX_ERR_ALIGN;
+    if (in_dtype != PARALLAX_BF16 || (out_dtype != PARALLAX_F32 && out_dtype != PARALLAX_BF16))
+        return PARALLAX_ERR_DTYPE;
+    DevState *s = nullptr;
+    int st = get_state(&s);
+    if (st) return st;
+    const DecodePlan plan = plan_decode(B, H, Tcap, d, s->sms);
+    void *ws = nullptr;
+    CallScratch scratch(s, static_cast<cudaStream_t>(stream));
+    if ((st = scratch.get(decode_partials_bytes(B, H, d, plan), &ws))) return st;
+    return status_of(launch_softmax_decode(q, kcache, vcache, seqlens, y, lse, B, H, Tcap, d, out_dtype, plan,
+                                           static_cast<float *>(ws), static_cast<cudaStream_t>(stream)));
+}
+
 int parallax_decode_paged(const void *q, const void *rho, const void *kpages, const void *vpages,
                           const int *block_table, const int *seqlens, void *y, float *lse, int B, int Hq, int Hkv,
                           int page_size, int max_pages, int num_pages, int d, int in_dtype, int out_dtype,

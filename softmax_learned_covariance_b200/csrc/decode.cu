@@ -82,7 +82,9 @@ template <int D> struct DecodeSmem {
     float red_s[3][NW];
 };
 
-template <int D, typename Tout>
+// WITH_RHO = false: plain softmax attention decode (no probe, no correction
+// branch) -- the reference point the pages compare the Parallax decode with.
+template <int D, typename Tout, bool WITH_RHO = true>
 __global__ void __launch_bounds__(NTHREADS, MIN_BLOCKS) k_decode_split(
     const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ rho, const __nv_bfloat16 *__restrict__ kc,
     const __nv_bfloat16 *__restrict__ vc, const int *__restrict__ seqlens, Tout *__restrict__ y,
@@ -111,9 +113,14 @@ __global__ void __launch_bounds__(NTHREADS, MIN_BLOCKS) k_decode_split(
         float qv[8], rv[8];
         {
             const uint4 *qp = reinterpret_cast<const uint4 *>(q + bh * D) + c;
-            const uint4 *rp = reinterpret_cast<const uint4 *>(rho + bh * D) + c;
             unpack8(__ldg(qp), qv);
-            unpack8(__ldg(rp), rv);
+            if constexpr (WITH_RHO) {
+                const uint4 *rp = reinterpret_cast<const uint4 *>(rho + bh * D) + c;
+                unpack8(__ldg(rp), rv);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) rv[e] = 0.f;
+            }
         }
         const uint4 *kbase = reinterpret_cast<const uint4 *>(kc + (size_t)bh * Tcap * D) + c;
         const uint4 *vbase = reinterpret_cast<const uint4 *>(vc + (size_t)bh * Tcap * D) + c;
@@ -141,12 +148,12 @@ __global__ void __launch_bounds__(NTHREADS, MIN_BLOCKS) k_decode_split(
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         dz = fmaf(qv[e], kf[e], dz);
-                        da = fmaf(rv[e], kf[e], da);
+                        if constexpr (WITH_RHO) da = fmaf(rv[e], kf[e], da);
                     }
 #pragma unroll
                     for (int off = LPT / 2; off > 0; off >>= 1) {
                         dz += __shfl_xor_sync(0xffffffffu, dz, off);
-                        da += __shfl_xor_sync(0xffffffffu, da, off);
+                        if constexpr (WITH_RHO) da += __shfl_xor_sync(0xffffffffu, da, off);
                     }
                     const int tok = base + x * GROUPS + slot;
                     if (c == 0 && tok < n) {
@@ -203,7 +210,7 @@ __global__ void __launch_bounds__(NTHREADS, MIN_BLOCKS) k_decode_split(
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
                             O[e] = fmaf(p, vf[e], O[e]);
-                            M[e] = fmaf(pa, vf[e], M[e]);
+                            if constexpr (WITH_RHO) M[e] = fmaf(pa, vf[e], M[e]);
                         }
                     }
                 }
@@ -351,20 +358,24 @@ __global__ void __launch_bounds__(CMB_WARPS * 32) k_decode_combine(const float *
         red[warp][2 * D + 1] = ab;
     }
     __syncthreads();
-    if (tid < D) {
-        float lt = 0.f, at = 0.f, ot = 0.f, mt = 0.f;
+    float lt = 0.f, at = 0.f;
+#pragma unroll
+    for (int w = 0; w < CMB_WARPS; ++w) {
+        lt += red[w][2 * D];
+        at += red[w][2 * D + 1];
+    }
+    const float inv = 1.0f / lt;
+    for (int e = tid; e < D; e += CMB_WARPS * 32) {   // one output dimension per thread
+        float ot = 0.f, mt = 0.f;
 #pragma unroll
         for (int w = 0; w < CMB_WARPS; ++w) {
-            lt += red[w][2 * D];
-            at += red[w][2 * D + 1];
-            ot += red[w][tid];
-            mt += red[w][D + tid];
+            ot += red[w][e];
+            mt += red[w][D + e];
         }
-        const float inv = 1.0f / lt;
         const float oo = ot * inv;
-        store_out<Tout>(y + bh * D + tid, oo - (mt * inv - oo * (at * inv)));
-        if (lse != nullptr && tid == 0) lse[bh] = (mu + log2f(lt)) * LN2;
+        store_out<Tout>(y + bh * D + e, oo - (mt * inv - oo * (at * inv)));
     }
+    if (lse != nullptr && tid == 0) lse[bh] = (mu + log2f(lt)) * LN2;
 }
 
 template <int D, typename Tout>
@@ -379,13 +390,13 @@ cudaError_t launch_combine(const float *partials, const int *seqlens, void *y, f
     return cudaGetLastError();
 }
 
-template <int D, typename Tout>
+template <int D, typename Tout, bool WITH_RHO = true>
 cudaError_t launch_t(const void *q, const void *rho, const void *kc, const void *vc, const int *seqlens, void *y,
                      float *lse, int B, int H, int Tcap, const DecodePlan &p, float *partials, cudaStream_t s) {
     const long BH = (long)B * H;
     const long units = BH * p.nsplit;
     const long grid = units < 0x7fffffffL ? units : 0x7fffffffL;   // one CTA per unit
-    k_decode_split<D, Tout><<<(unsigned)grid, NTHREADS, 0, s>>>(
+    k_decode_split<D, Tout, WITH_RHO><<<(unsigned)grid, NTHREADS, 0, s>>>(
         (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)rho, (const __nv_bfloat16 *)kc, (const __nv_bfloat16 *)vc,
         seqlens, (Tout *)y, lse, H, Tcap, p.chunk, p.nsplit, BH, partials);
     cudaError_t e = cudaGetLastError();
@@ -408,6 +419,21 @@ cudaError_t launch_decode(const void *q, const void *rho, const void *kc, const 
     if (out_dtype == PARALLAX_F32)
         return launch_t<128, float>(q, rho, kc, vc, seqlens, y, lse, B, H, Tcap, p, partials, s);
     return launch_t<128, __nv_bfloat16>(q, rho, kc, vc, seqlens, y, lse, B, H, Tcap, p, partials, s);
+}
+
+cudaError_t launch_softmax_decode(const void *q, const void *kc, const void *vc, const int *seqlens, void *y,
+                                  float *lse, int B, int H, int Tcap, int d, int out_dtype, const DecodePlan &p,
+                                  float *partials, cudaStream_t s) {
+    const bool f32 = out_dtype == PARALLAX_F32;
+    if (d == 64)
+        return f32 ? launch_t<64, float, false>(q, nullptr, kc, vc, seqlens, y, lse, B, H, Tcap, p, partials, s)
+                   : launch_t<64, __nv_bfloat16, false>(q, nullptr, kc, vc, seqlens, y, lse, B, H, Tcap, p, partials, s);
+    if (d == 128)
+        return f32 ? launch_t<128, float, false>(q, nullptr, kc, vc, seqlens, y, lse, B, H, Tcap, p, partials, s)
+                   : launch_t<128, __nv_bfloat16, false>(q, nullptr, kc, vc, seqlens, y, lse, B, H, Tcap, p, partials,
+                                                         s);
+    return f32 ? launch_t<256, float, false>(q, nullptr, kc, vc, seqlens, y, lse, B, H, Tcap, p, partials, s)
+               : launch_t<256, __nv_bfloat16, false>(q, nullptr, kc, vc, seqlens, y, lse, B, H, Tcap, p, partials, s);
 }
 
 cudaError_t launch_decode_paged(const void *q, const void *rho, const void *kpages, const void *vpages,

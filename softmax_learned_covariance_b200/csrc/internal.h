@@ -43,6 +43,12 @@ cudaError_t launch_decode(const void *q, const void *rho, const void *kc, const 
                           void *y, float *lse, int B, int H, int Tcap, int d, int out_dtype, const DecodePlan &p,
                           float *partials, int sm_count, const DeviceCtl &ctl, cudaStream_t s);
 
+// Plain softmax attention decode (no probe) with the same split kernel, d in
+// {64, 128, 256}: the reference point the pages compare the decode with.
+cudaError_t launch_softmax_decode(const void *q, const void *kc, const void *vc, const int *seqlens, void *y,
+                                  float *lse, int B, int H, int Tcap, int d, int out_dtype, const DecodePlan &p,
+                                  float *partials, cudaStream_t s);
+
 // Paged KV layout for the decode: pages [num_pages, Hkv, 1 << pshift, d];
 // query head h reads KV head h / group.
 struct PagedKV {

@@ -91,6 +91,16 @@ def test_decode_host_validation(L):
     assert dec(o=7) == 4
 
 
+def test_softmax_decode_host_validation(L):
+    def sd(q=A16, kc=A16, vc=A16, sl=A16, y=A16, Tcap=16, d=256, i=1, o=0):
+        return L.parallax_softmax_decode(q, kc, vc, sl, y, None, 2, 2, Tcap, d, i, o, None)
+    assert sd(kc=None) == 1
+    assert sd(d=96) == 2
+    assert sd(Tcap=0) == 2
+    assert sd(vc=MIS) == 3
+    assert sd(i=0) == 4
+
+
 def test_decode_paged_host_validation(L):
     def dec(q=A16, rho=A16, kp=A16, vp=A16, bt=A16, sl=A16, y=A16, B=2, Hq=4, Hkv=2, ps=64, mp=4, npg=8, d=128,
             i=1, o=0):

@@ -108,3 +108,26 @@ def test_long_context_cells_sampled_heads(B, ctx):
         yr, lr = oracle.decode(hq.f64, hr.f64, hk.f64, hv.f64, sl[b:b + 1])
         parity.assert_bf16_parity(y[b:b + 1, h:h + 1].cpu().numpy(), yr, 2, f"B={B} ctx={ctx} head {b},{h}")
         parity.assert_lse(lse[b:b + 1, h:h + 1].cpu().numpy(), lr)
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_softmax_decode_reference(d):
+    """parallax_softmax_decode (the pages' comparison baseline) against the oracle
+    at rho = 0 (softmax attention), ragged lengths including 1 and Tcap; at
+    d 64 / 128 it is bitwise parallax_decode with rho = 0 (same split, same sums)."""
+    B, H, Tcap = 6, 4, 3000
+    sl = np.array([1, 17, 1500, 2999, 3000, 256], np.int32)
+    q, rho, kc, vc, _ = inputs.decode_inputs(B, H, Tcap, d, seqlens=sl, seed=700 + d)
+    dq, dk, dv = q.torch().to(DEV), kc.torch().to(DEV), vc.torch().to(DEV)
+    ds = torch.from_numpy(sl).to(DEV)
+    y, lse = plx.parallax_softmax_decode(dq, dk, dv, ds)
+    torch.cuda.synchronize()
+    assert plx.parallax_last_device_error() == 0
+    zero = np.zeros_like(rho.f64)
+    yr, lr = oracle.decode(q.f64, zero, kc.f64, vc.f64, sl)
+    parity.assert_bf16_parity(y.cpu().numpy(), yr, 2, f"softmax decode d={d}")
+    parity.assert_lse(lse.cpu().numpy(), lr)
+    if d != 256:
+        y0, l0 = plx.parallax_decode(dq, torch.zeros_like(rho.torch().to(DEV)), dk, dv, ds)
+        torch.cuda.synchronize()
+        assert torch.equal(y0, y) and torch.equal(l0, lse)
