@@ -11,14 +11,16 @@
 // ordered chunk-major: every head's first chunks (full length for any ragged
 // mix) come first and the short or empty tails last, so the hardware block
 // scheduler balances ragged sequence lengths without a host-side read of
-// seqlens.  16 resident CTAs (32 warps) per SM keep enough 16-byte loads in
-// flight to cover HBM latency.  Within a unit the tokens are taken in
-// sub-chunks of SUB: pass A streams K with 16-byte loads (one token row per
-// D/8 lanes, fully coalesced) and stages z, a in shared memory; the sub-chunk
-// max updates the running max (one rescale per sub-chunk, not per token);
-// pass B streams V and accumulates o and m in fp32.  A unit writes either the
-// final y (one unit per sequence) or its partial state (mu, l, abar, O, M) for
-// the combine kernel, which merges the partials with max-rescaling.
+// seqlens.  Within a unit each token row is read by D/8 lanes (16 bytes each,
+// fully coalesced); a warp holds 32/(D/8) rows at a time and a lane group
+// keeps its own online-softmax state over the rows it reads: per step it loads
+// the K and V rows of UNF tokens together, forms z and a from the K row, moves
+// its reference max only when a score exceeds it by more than 2^8 (so the
+// rescale of its accumulators is rare), and accumulates o and m from the V
+// row.  The lane groups' states meet once per unit in shared memory.  A unit
+// writes either the final y (one unit per sequence) or its partial state
+// (mu, l, abar, O, M) for the combine kernel, which merges the partials with
+// max-rescaling.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -27,18 +29,25 @@
 namespace plx {
 namespace {
 
-// Measured on B200 (bench shape B=64 H=16 ctx 4096): 2-warp CTAs with 16 of them
-// resident per SM (64 registers per thread) stream at 5.3-5.5 TB/s across runs,
-// 4-warp CTAs at 8 per SM at 5.1-5.26 TB/s, 8-warp CTAs at 3 per SM at 4.4-4.5
-// TB/s, and a TMA-ring variant whose consumer warps were latency bound per block
-// at 3.6-3.8 TB/s.
-// Small CTAs keep the __syncthreads-separated phases of one CTA from idling the
-// SM: the other CTAs' loads are in flight meanwhile.
+// Measured on B200 (bench shape B=64 H=16 ctx 4096, CUDA events):
+// * one pass with K and V rows loaded together and per-lane-group softmax
+//   state, 4 tokens per lane group in flight, 2-warp CTAs at 12 per SM (80
+//   registers): 0.31 ms, within 2 % of the softmax-only instantiation;
+// * the same with 2 tokens in flight: 0.34 ms; with 8 tokens at 8 CTAs per SM,
+//   or 4-warp CTAs: within 2 % of the 4-token form, slower on short caches;
+// * two passes per 512-token sub-chunk (K pass staging z and a in shared
+//   memory, block max, V pass), 16 CTAs per SM: 0.38 ms -- the barrier-separated
+//   phases left loads idle while the Parallax arithmetic ran, 17 % behind the
+//   softmax-only instantiation of the same code;
+// * 8-warp CTAs or a TMA-ring variant: 0.47-0.6 ms.
+// The K dot products take bf16 operands straight from the loaded words
+// (mixed-precision fma with f32 accumulation: exact products, as after a
+// widening), which saves the unpacking of K and keeps q and rho packed.
 constexpr int NW = 2;            // warps per CTA
 constexpr int NTHREADS = NW * 32;
-constexpr int SUB = 512;         // tokens staged per sub-chunk
-constexpr int UNROLL = 4;        // 16-byte loads in flight per lane per pass step
-constexpr int MIN_BLOCKS = 16;   // resident CTAs per SM the register budget targets
+constexpr int UNF = 4;           // tokens a lane group has in flight per step (K and V rows)
+constexpr int MIN_BLOCKS = 12;   // resident CTAs per SM the register budget targets
+constexpr float RESCALE_LOG2 = 8.0f;   // reference max moves when a score exceeds it by this
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 
@@ -71,16 +80,32 @@ template <> __device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat
     *p = __float2bfloat16_rn(v);
 }
 
-template <int D> struct DecodeSmem {
-    static constexpr int LPT = D / 8;        // lanes per token row
-    static constexpr int TPW = 32 / LPT;     // token rows per warp step
-    static constexpr int GROUPS = NW * TPW;  // token slots per CTA step
-    float z[SUB];                            // scores (log2 units), then p
-    float a[SUB];                            // a_j, then p_j a_j
-    float red_o[GROUPS][D];
-    float red_m[GROUPS][D];
-    float red_s[3][NW];
-};
+// c + a.b with a, b the low (hi = false) or high bf16 halves of two packed
+// words, f32 accumulation (the product of two bf16 values is exact in f32).
+__device__ __forceinline__ float fma_bf16_half(uint32_t a, uint32_t b, float c, bool hi) {
+    float r;
+    if (hi)
+        asm("{.reg .b16 al, ah, bl, bh;\n mov.b32 {al, ah}, %1;\n mov.b32 {bl, bh}, %2;\n"
+            " fma.rn.f32.bf16 %0, ah, bh, %3;\n}"
+            : "=f"(r) : "r"(a), "r"(b), "f"(c));
+    else
+        asm("{.reg .b16 al, ah, bl, bh;\n mov.b32 {al, ah}, %1;\n mov.b32 {bl, bh}, %2;\n"
+            " fma.rn.f32.bf16 %0, al, bl, %3;\n}"
+            : "=f"(r) : "r"(a), "r"(b), "f"(c));
+    return r;
+}
+
+// Dot product of 8 packed bf16 values with 8 others, f32 accumulation.
+__device__ __forceinline__ float dot8_bf16(const uint4 &x, const uint4 &k) {
+    const uint32_t xw[4] = {x.x, x.y, x.z, x.w}, kw[4] = {k.x, k.y, k.z, k.w};
+    float acc = 0.f;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        acc = fma_bf16_half(xw[t], kw[t], acc, false);
+        acc = fma_bf16_half(xw[t], kw[t], acc, true);
+    }
+    return acc;
+}
 
 // WITH_RHO = false: plain softmax attention decode (no probe, no correction
 // branch) -- the reference point the pages compare the Parallax decode with.
@@ -89,15 +114,18 @@ __global__ void __launch_bounds__(NTHREADS, MIN_BLOCKS) k_decode_split(
     const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ rho, const __nv_bfloat16 *__restrict__ kc,
     const __nv_bfloat16 *__restrict__ vc, const int *__restrict__ seqlens, Tout *__restrict__ y,
     float *__restrict__ lse, int H, int Tcap, int chunk, int nsplit, long BH, float *__restrict__ partials) {
-    using S = DecodeSmem<D>;
-    constexpr int LPT = S::LPT, TPW = S::TPW, GROUPS = S::GROUPS;
-    constexpr int STEP = GROUPS * UNROLL;    // token rows per unrolled step
-    __shared__ S sm;
+    constexpr int LPT = D / 8;               // lanes per token row
+    constexpr int TPW = 32 / LPT;            // token rows per warp
+    constexpr int GROUPS = NW * TPW;         // lane groups (token slots) per CTA
+    constexpr int STEP = GROUPS * UNF;       // token rows per CTA step
+    __shared__ float red_o[GROUPS][D];
+    __shared__ float red_m[GROUPS][D];
+    __shared__ float red_s[3][GROUPS];
 
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-    const int g = lane / LPT;                 // token slot within the warp
+    const int g = lane / LPT;                 // lane group within the warp
     const int c = lane % LPT;                 // 16-byte column within the row
-    const int slot = warp * TPW + g;          // token slot within the CTA step
+    const int slot = warp * TPW + g;          // lane group within the CTA
     const float scale_log2 = LOG2E / sqrtf((float)D);
 
     const long units = BH * nsplit;
@@ -110,136 +138,95 @@ __global__ void __launch_bounds__(NTHREADS, MIN_BLOCKS) k_decode_split(
         if (t0 >= L && nsplit > 1) continue;  // beyond this sequence: no partial
         const int t1 = min(L, t0 + chunk);
 
-        float qv[8], rv[8];
-        {
-            const uint4 *qp = reinterpret_cast<const uint4 *>(q + bh * D) + c;
-            unpack8(__ldg(qp), qv);
-            if constexpr (WITH_RHO) {
-                const uint4 *rp = reinterpret_cast<const uint4 *>(rho + bh * D) + c;
-                unpack8(__ldg(rp), rv);
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) rv[e] = 0.f;
-            }
-        }
+        const uint4 qp = __ldg(reinterpret_cast<const uint4 *>(q + bh * D) + c);
+        uint4 rp = make_uint4(0, 0, 0, 0);
+        if constexpr (WITH_RHO) rp = __ldg(reinterpret_cast<const uint4 *>(rho + bh * D) + c);
         const uint4 *kbase = reinterpret_cast<const uint4 *>(kc + (size_t)bh * Tcap * D) + c;
         const uint4 *vbase = reinterpret_cast<const uint4 *>(vc + (size_t)bh * Tcap * D) + c;
 
-        float mu = -INFINITY, lsum = 0.f, asum = 0.f;
+        // this lane group's state: reference max (log2 units), sums, and its 8 columns of O, M
+        float mref = -INFINITY, lsum = 0.f, asum = 0.f;
         float O[8], M[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) O[e] = M[e] = 0.f;
 
-        for (int s0 = t0; s0 < t1; s0 += SUB) {
-            const int n = min(SUB, t1 - s0);
-            // ---- pass A: K stream -> z (log2 units) and a ----
-            for (int base = 0; base < n; base += STEP) {
-                uint4 kr[UNROLL];
+        for (int base = t0; base < t1; base += STEP) {
+            uint4 kr[UNF], vr[UNF];
 #pragma unroll
-                for (int x = 0; x < UNROLL; ++x) {
-                    const int tok = base + x * GROUPS + slot;
-                    kr[x] = tok < n ? ldg_stream(kbase + (size_t)(s0 + tok) * LPT) : make_uint4(0, 0, 0, 0);
+            for (int x = 0; x < UNF; ++x) {
+                const int tok = base + x * GROUPS + slot;
+                const bool ok = tok < t1;
+                kr[x] = ok ? ldg_stream(kbase + (size_t)tok * LPT) : make_uint4(0, 0, 0, 0);
+                vr[x] = ok ? ldg_stream(vbase + (size_t)tok * LPT) : make_uint4(0, 0, 0, 0);
+            }
+            float z[UNF], a[UNF];
+            float bm = -INFINITY;
+#pragma unroll
+            for (int x = 0; x < UNF; ++x) {
+                float dz = dot8_bf16(qp, kr[x]);
+                float da = 0.f;
+                if constexpr (WITH_RHO) da = dot8_bf16(rp, kr[x]);
+                // butterfly over the row's lanes: every lane ends with the same sums
+#pragma unroll
+                for (int off = LPT / 2; off > 0; off >>= 1) {
+                    dz += __shfl_xor_sync(0xffffffffu, dz, off);
+                    if constexpr (WITH_RHO) da += __shfl_xor_sync(0xffffffffu, da, off);
                 }
+                const int tok = base + x * GROUPS + slot;
+                z[x] = tok < t1 ? dz * scale_log2 : -INFINITY;
+                a[x] = da;
+                bm = fmaxf(bm, z[x]);
+            }
+            if (bm > mref + RESCALE_LOG2) {   // the same decision in every lane of the group
+                const float alpha = fex2(mref - bm);   // 0 while mref = -inf
+                mref = bm;
+                lsum *= alpha;
+                asum *= alpha;
 #pragma unroll
-                for (int x = 0; x < UNROLL; ++x) {
-                    float kf[8];
-                    unpack8(kr[x], kf);
-                    float dz = 0.f, da = 0.f;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        dz = fmaf(qv[e], kf[e], dz);
-                        if constexpr (WITH_RHO) da = fmaf(rv[e], kf[e], da);
-                    }
-#pragma unroll
-                    for (int off = LPT / 2; off > 0; off >>= 1) {
-                        dz += __shfl_xor_sync(0xffffffffu, dz, off);
-                        if constexpr (WITH_RHO) da += __shfl_xor_sync(0xffffffffu, da, off);
-                    }
-                    const int tok = base + x * GROUPS + slot;
-                    if (c == 0 && tok < n) {
-                        sm.z[tok] = dz * scale_log2;
-                        sm.a[tok] = da;
-                    }
+                for (int e = 0; e < 8; ++e) {
+                    O[e] *= alpha;
+                    M[e] *= alpha;
                 }
             }
-            __syncthreads();
-            // ---- sub-chunk max, running rescale ----
-            float mx = -INFINITY;
-            for (int t = tid; t < n; t += NTHREADS) mx = fmaxf(mx, sm.z[t]);
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-            if (lane == 0) sm.red_s[0][warp] = mx;
-            __syncthreads();
-            mx = sm.red_s[0][0];
-#pragma unroll
-            for (int w = 1; w < NW; ++w) mx = fmaxf(mx, sm.red_s[0][w]);
-            const float mu_new = fmaxf(mu, mx);
-            const float alpha = fex2(mu - mu_new);   // 0 when mu = -inf
-            mu = mu_new;
-            lsum *= alpha;
-            asum *= alpha;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                O[e] *= alpha;
-                M[e] *= alpha;
-            }
-            for (int t = tid; t < n; t += NTHREADS) {
-                const float p = fex2(sm.z[t] - mu);
-                const float pa = p * sm.a[t];
-                sm.z[t] = p;
-                sm.a[t] = pa;
+            for (int x = 0; x < UNF; ++x) {
+                const float p = z[x] == -INFINITY ? 0.f : fex2(z[x] - mref);
+                const float pa = p * a[x];
                 lsum += p;
                 asum += pa;
-            }
-            __syncthreads();
-            // ---- pass B: V stream -> O += p v, M += p a v ----
-            for (int base = 0; base < n; base += STEP) {
-                uint4 vr[UNROLL];
+                float vf[8];
+                unpack8(vr[x], vf);
 #pragma unroll
-                for (int x = 0; x < UNROLL; ++x) {
-                    const int tok = base + x * GROUPS + slot;
-                    vr[x] = tok < n ? ldg_stream(vbase + (size_t)(s0 + tok) * LPT) : make_uint4(0, 0, 0, 0);
-                }
-#pragma unroll
-                for (int x = 0; x < UNROLL; ++x) {
-                    const int tok = base + x * GROUPS + slot;
-                    if (tok < n) {
-                        float vf[8];
-                        unpack8(vr[x], vf);
-                        const float p = sm.z[tok], pa = sm.a[tok];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            O[e] = fmaf(p, vf[e], O[e]);
-                            if constexpr (WITH_RHO) M[e] = fmaf(pa, vf[e], M[e]);
-                        }
-                    }
+                for (int e = 0; e < 8; ++e) {
+                    O[e] = fmaf(p, vf[e], O[e]);
+                    if constexpr (WITH_RHO) M[e] = fmaf(pa, vf[e], M[e]);
                 }
             }
-            __syncthreads();
         }
 
-        // ---- reduce over token slots and threads ----
+        // ---- merge the lane groups: common reference max mu, then the sums ----
+        if (c == 0) red_s[0][slot] = mref;
+        __syncthreads();
+        float mu = red_s[0][0];
+#pragma unroll
+        for (int s = 1; s < GROUPS; ++s) mu = fmaxf(mu, red_s[0][s]);
+        const float w = mref == -INFINITY ? 0.f : fex2(mref - mu);   // a group that read no token adds 0
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-            sm.red_o[slot][c * 8 + e] = O[e];
-            sm.red_m[slot][c * 8 + e] = M[e];
+            red_o[slot][c * 8 + e] = O[e] * w;
+            red_m[slot][c * 8 + e] = M[e] * w;
         }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
-            asum += __shfl_xor_sync(0xffffffffu, asum, off);
-        }
-        if (lane == 0) {
-            sm.red_s[1][warp] = lsum;
-            sm.red_s[2][warp] = asum;
+        if (c == 0) {
+            red_s[1][slot] = lsum * w;
+            red_s[2][slot] = asum * w;
         }
         __syncthreads();
         {
             float l = 0.f, ab = 0.f;
 #pragma unroll
-            for (int w = 0; w < NW; ++w) {
-                l += sm.red_s[1][w];
-                ab += sm.red_s[2][w];
+            for (int s = 0; s < GROUPS; ++s) {
+                l += red_s[1][s];
+                ab += red_s[2][s];
             }
             float *P = partials + ((size_t)bh * nsplit + split) * (2 * D + 3);
             // one output dimension per thread, striding when the CTA is narrower than d
@@ -247,8 +234,8 @@ __global__ void __launch_bounds__(NTHREADS, MIN_BLOCKS) k_decode_split(
                 float o = 0.f, m = 0.f;
 #pragma unroll
                 for (int s = 0; s < GROUPS; ++s) {
-                    o += sm.red_o[s][e];
-                    m += sm.red_m[s][e];
+                    o += red_o[s][e];
+                    m += red_m[s][e];
                 }
                 if (nsplit == 1) {
                     float out = 0.f;
@@ -273,7 +260,7 @@ __global__ void __launch_bounds__(NTHREADS, MIN_BLOCKS) k_decode_split(
                 }
             }
         }
-        __syncthreads();
+        __syncthreads();   // the shared arrays are reused by the next unit
     }
 }
 
