@@ -70,6 +70,7 @@
 
 #include "internal.h"
 #include "sm100.cuh"
+#include "softmax_sm100.cuh"
 
 namespace plx {
 namespace {
@@ -110,11 +111,14 @@ template <int D> struct Geo {
     static_assert(OCOLS % 16 == 0, "16-column TMEM loads");
 };
 
-// TMEM column map.  S(j) and then A(j) land in X.  Group g writes its fp16 P
-// (16 columns) and P o A' (16 columns) to [COL_P + 32g, +32).  O and M start
-// on 128-column boundaries for both head dims.
-constexpr uint32_t COL_X = 0, COL_P = 128, COL_O = 256, COL_M = 384;
-__host__ __device__ constexpr uint32_t col_p(uint32_t kk) { return COL_P + (kk >> 1) * GCOLS + (kk & 1) * 8; }
+// TMEM column map: two tile regions X0, X1 and the accumulators O, M' (on
+// 128-column boundaries for both head dims).  Key tile G of the CTA uses
+// region X(G & 1): S(G) lands there, then A(G), and group g writes its fp16 P
+// (16 columns) and P o A' (16 columns) over [32g, 32g + 32) of the region --
+// the S and A columns it has already read -- where the P.V UMMAs read them.
+constexpr uint32_t COL_X0 = 0, COL_O = 256, COL_M = 384;
+__host__ __device__ constexpr uint32_t col_x(uint32_t G) { return COL_X0 + (G & 1) * BN; }
+__host__ __device__ constexpr uint32_t col_p(uint32_t kk) { return (kk >> 1) * GCOLS + (kk & 1) * 8; }
 constexpr uint32_t PA_SHIFT = GCOLS / 2;   // P o A' sits 16 columns after P
 
 constexpr uint32_t IDESC_S = idesc_f16(1, 1, 0, 0, BM, BN);     // bf16 Q/R (K-major) x bf16 K (K-major)
@@ -126,9 +130,9 @@ struct __align__(8) Bars {
     uint64_t k_full[KST], k_empty[KST];
     uint64_t v_full[VST], v_empty[VST];
     uint64_t s_full, a_full;      // S, A UMMAs of the current tile done
-    uint64_t s_free, a_free;      // softmax has loaded S, A out of TMEM
-    uint64_t p_full;              // P and P o A' are in TMEM
-    uint64_t pv_done;             // P.V UMMAs of the tile done
+    uint64_t s_free;              // softmax has loaded S out of TMEM
+    uint64_t p_full[2];           // per region: P and P o A' of its tile are in TMEM
+    uint64_t pv_done[2];          // per region: P.V UMMAs of its tile done
     uint64_t om_free;             // epilogue has read O and M
     uint64_t xchg[2];             // per tile parity: every softmax warp posted its partial max
     uint64_t esum;                // per item: partial sums posted
@@ -155,73 +159,6 @@ __device__ __forceinline__ Item item_of(int w, int BH, int nq, int T, int causal
     const int kend = causal ? min(T, (it.qt + 1) * BM) : T;
     it.nkv = (kend + BN - 1) / BN;
     return it;
-}
-
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-    float r;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-    return r;
-}
-
-// Bounded wait whose outcome is the same for all 32 lanes (lanes that saw the
-// phase complete still give up if another lane of the warp gave up), so the
-// .sync.aligned tcgen05 instructions that follow are never reached divergently.
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const WaitCtl &wc) {
-    const bool got = mbar_wait(bar, parity, wc);
-    return __all_sync(0xffffffffu, got);
-}
-
-// Everyone but the scheduler takes the k-th scheduled item from the ring.
-__device__ __forceinline__ bool next_item(Bars *bars, uint32_t k, int &w, const WaitCtl &wc) {
-    const uint32_t s = k % SCHED;
-    if (!mbar_wait(smem_u32(&bars->sched_full[s]), (k / SCHED) & 1, wc)) return false;
-    w = bars->sched_item[s];
-    return true;
-}
-
-// d0,d1 = a0,a1 * b + c as one packed fp32x2 FMA.
-__device__ __forceinline__ void ffma2(float &d0, float &d1, float a0, float a1, float b, float c) {
-    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %4};\n\tmov.b64 rc, {%5, %5};\n\t"
-        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d0), "=f"(d1)
-        : "f"(a0), "f"(a1), "f"(b), "f"(c));
-}
-
-// d = a * b + c elementwise on two fp32 pairs (one packed FMA).
-__device__ __forceinline__ void fma2v(float &d0, float &d1, float a0, float a1, float b0, float b1, float c0,
-                                      float c1) {
-    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d0), "=f"(d1)
-        : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
-}
-
-// 2^x for a pair on the FMA pipe.  The special-function unit does 16
-// exponentials per clock per SM, which bounds the softmax; a share of them is
-// taken here instead.  Range reduction: j = round(x) is read from the low
-// mantissa bits of x + 1.5 * 2^23, f = x - j lies in [-1/2, 1/2], and 2^f is a
-// degree-3 polynomial whose coefficients are the relative-error minimax fit on
-// [-1/2, 1/2] from a Remez exchange (max relative error 7.5e-5, well under the
-// fp16 rounding of P).  2^j is added to the exponent field.  x is clamped at
-// -125 so the exponent stays normal; results there (and for x = -inf) are
-// below 2^-124 and round to 0 in fp16.
-constexpr float EXP2_C0 = 0.99992806f, EXP2_C1 = 0.69326097f, EXP2_C2 = 0.24261113f, EXP2_C3 = 0.05517167f;
-__device__ __forceinline__ void exp2_poly2(float &y0, float &y1, float x0, float x1) {
-    constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
-    x0 = fmaxf(x0, -125.0f);
-    x1 = fmaxf(x1, -125.0f);
-    float t0, t1, r0, r1, f0, f1, p0, p1;
-    ffma2(t0, t1, x0, x1, 1.0f, kRound);    // kRound + round(x)
-    ffma2(r0, r1, t0, t1, 1.0f, -kRound);   // round(x), exact
-    fma2v(f0, f1, r0, r1, -1.0f, -1.0f, x0, x1);
-    fma2v(p0, p1, f0, f1, EXP2_C3, EXP2_C3, EXP2_C2, EXP2_C2);
-    fma2v(p0, p1, p0, p1, f0, f1, EXP2_C1, EXP2_C1);
-    fma2v(p0, p1, p0, p1, f0, f1, EXP2_C0, EXP2_C0);
-    // bits(t) << 23 == round(x) << 23 (mod 2^32): the low 9 bits of bits(1.5 * 2^23) are zero
-    y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-    y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
 template <int D, bool WITH_RHO, bool FUSED, typename Tout>
@@ -266,9 +203,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_init(smem_u32(&bars->s_full), 1);
         mbar_init(smem_u32(&bars->a_full), 1);
         mbar_init(smem_u32(&bars->s_free), NSOFT_WARPS);
-        mbar_init(smem_u32(&bars->a_free), NSOFT_WARPS);
-        mbar_init(smem_u32(&bars->p_full), NSOFT_WARPS);
-        mbar_init(smem_u32(&bars->pv_done), 1);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(smem_u32(&bars->p_full[x]), NSOFT_WARPS);
+            mbar_init(smem_u32(&bars->pv_done[x]), 1);
+        }
         mbar_init(smem_u32(&bars->om_free), NSOFT_WARPS);
         mbar_init(smem_u32(&bars->xchg[0]), NSOFT_WARPS);
         mbar_init(smem_u32(&bars->xchg[1]), NSOFT_WARPS);
@@ -374,7 +312,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         bool ok = true;
         for (uint32_t ic = 0; ok; ++ic) {
             int w;
-            if (!next_item(bars, ic, w, wc)) break;
+            if (!next_item<SCHED>(bars, ic, w, wc)) break;
             mbar_arrive(smem_u32(&bars->sched_empty[ic % SCHED]));
             if (w >= items) break;
             const Item it = item_of(w, BH, nq, T, causal);
@@ -397,9 +335,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (v_armed[s] >= 0) mbar_wait_drain(smem_u32(&bars->v_full[s]), (uint32_t)v_armed[s], DRAIN_NS);
     } else if (warp == 1 && lane == 0) {
         // ============================================= score UMMA issuer ==
-        // Per key tile j: S(j) into X once the softmax has loaded A(j-1)
-        // (S(j-1) without the correction branch), then A(j) into X once it
-        // has loaded S(j).  The shared-memory descriptors are built once; each
+        // Key tile G: S(G) into region X(G & 1) once the P.V UMMAs of tile
+        // G - 2 (the region's previous tile) are done, then A(G) there once the
+        // softmax has loaded S(G).  The shared-memory descriptors are built once; each
         // UMMA adds a compile-time offset, keeping this thread's instruction
         // stream short.
         uint32_t kc = 0, G = 0;
@@ -409,40 +347,42 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint64_t dk = sdesc_sw128(sbase + Gm::OFF_K, 16, 1024);   // stage s: + s * K_BYTES / 16
         // fused probe: R[128 x d] += X chunk (K-major) x W_R chunk (MN-major) into the P region
         constexpr uint32_t IDESC_R = idesc_f16(1, 1, 0, 1, BM, D);
-        auto issue_probe_chunk = [&](uint32_t stage_addr, bool first) {
+        auto issue_probe_chunk = [&](uint32_t dcol, uint32_t stage_addr, bool first) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
                 const uint64_t adesc = sdesc_sw128(stage_addr + kk * 32, 16, 1024);
                 const uint64_t bdesc = sdesc_sw128(stage_addr + XC_BYTES + kk * 16 * 128, 64 * 128, 1024);
-                umma_ss(tmem + COL_P, adesc, bdesc, IDESC_R, (first && kk == 0) ? 0u : 1u);
+                umma_ss(tmem + dcol, adesc, bdesc, IDESC_R, (first && kk == 0) ? 0u : 1u);
             }
         };
-        auto issue_scores = [&](uint64_t da, uint64_t kd) {
+        auto issue_scores = [&](uint32_t dcol, uint64_t da, uint64_t kd) {
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t off = ((uint32_t)(kk >> 2) * (Gm::Q_BYTES / Gm::HALVES) + (uint32_t)(kk & 3) * 32) >> 4;
                 const uint32_t koff =
                     ((uint32_t)(kk >> 2) * (Gm::K_BYTES / Gm::HALVES) + (uint32_t)(kk & 3) * 32) >> 4;
-                umma_ss(tmem + COL_X, da + off, kd + koff, IDESC_S, kk > 0 ? 1u : 0u);
+                umma_ss(tmem + dcol, da + off, kd + koff, IDESC_S, kk > 0 ? 1u : 0u);
             }
         };
         for (uint32_t ic = 0; ok; ++ic) {
             int w;
-            if (!next_item(bars, ic, w, wc)) break;
+            if (!next_item<SCHED>(bars, ic, w, wc)) break;
             mbar_arrive(smem_u32(&bars->sched_empty[ic % SCHED]));
             if (w >= items) break;
             const Item it = item_of(w, BH, nq, T, causal);
             if (!mbar_wait(smem_u32(&bars->qr_full), ic & 1, wc)) break;
             if constexpr (FUSED) {
-                // R of this item into the P region once the last P.V UMMAs of
-                // the previous item are done with it (this overlaps that item's
-                // epilogue, which reads O and M)
-                if (G > 0 && !mbar_wait(smem_u32(&bars->pv_done), (G - 1) & 1, wc)) break;
+                // R of this item into region X(G + 1) (that of the item's second
+                // tile) once the last P.V UMMAs of the previous item are done with
+                // it (this overlaps that item's epilogue, which reads O and M);
+                // S(G + 1) lands there only after A(G), which waits for the
+                // softmax to have moved R into shared memory
+                if (G > 0 && !mbar_wait(smem_u32(&bars->pv_done[(G - 1) & 1]), ((G - 1) >> 1) & 1, wc)) break;
                 for (int c = 0; c < nchunk; ++c, ++kc) {
                     const int s = kc % KST;
                     if (!mbar_wait(smem_u32(&bars->k_full[s]), (kc / KST) & 1, wc)) { ok = false; break; }
                     tc_fence_after();
-                    issue_probe_chunk(sbase + Gm::OFF_K + s * Gm::K_BYTES, c == 0);
+                    issue_probe_chunk(col_x(G + 1), sbase + Gm::OFF_K + s * Gm::K_BYTES, c == 0);
                     tc_commit(smem_u32(&bars->k_empty[s]));
                 }
                 if (!ok) break;
@@ -451,20 +391,27 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             for (int j = 0; j < it.nkv; ++j, ++G, ++kc) {
                 const int s = kc % KST;
                 if (!mbar_wait(smem_u32(&bars->k_full[s]), (kc / KST) & 1, wc)) { ok = false; break; }
-                if (G > 0 && !mbar_wait(smem_u32(WITH_RHO ? &bars->a_free : &bars->s_free), (G - 1) & 1, wc)) {
+                // the region's previous tile has been consumed by its P.V UMMAs
+                if (G >= 2 && !mbar_wait(smem_u32(&bars->pv_done[G & 1]), ((G - 2) >> 1) & 1, wc)) {
+                    ok = false;
+                    break;
+                }
+                // without the A UMMAs, nothing else orders S(G) after the
+                // softmax's load of S(G - 1), which keeps s_full one phase ahead
+                if (!WITH_RHO && G > 0 && !mbar_wait(smem_u32(&bars->s_free), (G - 1) & 1, wc)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const uint64_t kd = dk + (uint64_t)(s * (Gm::K_BYTES >> 4));
-                issue_scores(dq, kd);
+                issue_scores(col_x(G), dq, kd);
                 tc_commit(smem_u32(&bars->s_full));
                 if constexpr (WITH_RHO) {
                     // fused probe: the softmax warps have put R into shared memory
                     if (FUSED && j == 0 && !mbar_wait(smem_u32(&bars->r_smem), ic & 1, wc)) { ok = false; break; }
                     if (!mbar_wait(smem_u32(&bars->s_free), G & 1, wc)) { ok = false; break; }
                     tc_fence_after();
-                    issue_scores(dr, kd);
+                    issue_scores(col_x(G), dr, kd);
                     tc_commit(smem_u32(&bars->a_full));
                 }
                 tc_commit(smem_u32(&bars->k_empty[s]));
@@ -482,12 +429,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint64_t dv = sdesc_sw128(sbase + Gm::OFF_V, Gm::V_BYTES / Gm::HALVES, 1024);   // + s * V_BYTES / 16
         for (uint32_t ic = 0; ok; ++ic) {
             int w;
-            if (!next_item(bars, ic, w, wc)) break;
+            if (!next_item<SCHED>(bars, ic, w, wc)) break;
             mbar_arrive(smem_u32(&bars->sched_empty[ic % SCHED]));
             if (w >= items) break;
             const Item it = item_of(w, BH, nq, T, causal);
             for (int j = 0; j < it.nkv && ok; ++j, ++G) {
-                if (!mbar_wait(smem_u32(&bars->p_full), G & 1, wc)) { ok = false; break; }
+                if (!mbar_wait(smem_u32(&bars->p_full[G & 1]), (G >> 1) & 1, wc)) { ok = false; break; }
                 // the first tile overwrites O and M': the epilogue of the
                 // previous item must have read them
                 if (j == 0 && ic > 0 && !mbar_wait(smem_u32(&bars->om_free), (ic - 1) & 1, wc)) {
@@ -504,13 +451,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         const int kk = vs * (VKEYS / 16) + k2;     // 16-key step within the tile
                         const uint64_t vdesc = vd + (uint64_t)((k2 * 16 * 128) >> 4);
                         const uint32_t acc = (j == 0 && kk == 0) ? 0u : 1u;
-                        umma_ts(tmem + COL_O, tmem + col_p(kk), vdesc, IDESC_PV, acc);
-                        if constexpr (WITH_RHO)
-                            umma_ts(tmem + COL_M, tmem + col_p(kk) + PA_SHIFT, vdesc, IDESC_PV, acc);
+                        const uint32_t pc = tmem + col_x(G) + col_p(kk);
+                        umma_ts(tmem + COL_O, pc, vdesc, IDESC_PV, acc);
+                        if constexpr (WITH_RHO) umma_ts(tmem + COL_M, pc + PA_SHIFT, vdesc, IDESC_PV, acc);
                     }
                     tc_commit(smem_u32(&bars->v_empty[s]));
                 }
-                if (ok) tc_commit(smem_u32(&bars->pv_done));
+                if (ok) tc_commit(smem_u32(&bars->pv_done[G & 1]));
             }
         }
         tc_commit(smem_u32(&bars->drain[1]));
@@ -528,7 +475,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         bool ok = true;
         for (uint32_t ic = 0; ok; ++ic) {
             int w = 0;
-            const bool got = next_item(bars, ic, w, wc);
+            const bool got = next_item<SCHED>(bars, ic, w, wc);
             if (!__all_sync(0xffffffffu, got)) break;
             if (lane == 0) mbar_arrive(smem_u32(&bars->sched_empty[ic % SCHED]));
             if (w >= items) break;
@@ -537,17 +484,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int kvis = causal ? min(T, qrow + 1) : T;  // keys visible to this row
             float m_ref = -INFINITY, l = 0.f, ab = 0.f;
             if constexpr (FUSED) {
-                // ---- the probe tile R = X W_R of this item: TMEM (P region) ->
-                // bf16 -> shared memory, in the swizzled K-major layout a TMA
-                // load of rho would give, for the A UMMAs.  Group g converts
-                // columns [32g, 32g + 32) of its rows: the same TMEM columns it
-                // later overwrites with its P, so no group reads what another
-                // has already overwritten. ----
+                // ---- the probe tile R = X W_R of this item: TMEM (region
+                // X(G + 1)) -> bf16 -> shared memory, in the swizzled K-major
+                // layout a TMA load of rho would give, for the A UMMAs.  Group g
+                // converts columns [32g, 32g + 32) of its rows. ----
                 if (!warp_wait(smem_u32(&bars->r_tmem), ic & 1, wc)) { ok = false; break; }
                 tc_fence_after();
                 uint32_t rr[GCOLS];
-                tmem_ld16(tmem + lane_off + COL_P + grp * GCOLS, *reinterpret_cast<uint32_t(*)[16]>(&rr[0]));
-                tmem_ld16(tmem + lane_off + COL_P + grp * GCOLS + 16, *reinterpret_cast<uint32_t(*)[16]>(&rr[16]));
+                const uint32_t rcol = tmem + lane_off + col_x(G + 1) + grp * GCOLS;
+                tmem_ld16(rcol, *reinterpret_cast<uint32_t(*)[16]>(&rr[0]));
+                tmem_ld16(rcol + 16, *reinterpret_cast<uint32_t(*)[16]>(&rr[16]));
                 tmem_wait_ld();
                 uint8_t *rrow = smem + Gm::OFF_R + ((grp * GCOLS) / 64) * (Gm::Q_BYTES / Gm::HALVES) + r * 128;
 #pragma unroll
@@ -574,9 +520,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 // ---- scores of this group's 32 keys, then release S ----
                 if (!warp_wait(smem_u32(&bars->s_full), G & 1, wc)) { ok = false; break; }
                 tc_fence_after();
+                const uint32_t xcol = tmem + lane_off + col_x(G) + grp * GCOLS;   // this group's columns of the tile's region
                 uint32_t sr[GCOLS];
-                tmem_ld16(tmem + lane_off + COL_X + grp * GCOLS, *reinterpret_cast<uint32_t(*)[16]>(&sr[0]));
-                tmem_ld16(tmem + lane_off + COL_X + grp * GCOLS + 16, *reinterpret_cast<uint32_t(*)[16]>(&sr[16]));
+                tmem_ld16(xcol, *reinterpret_cast<uint32_t(*)[16]>(&sr[0]));
+                tmem_ld16(xcol + 16, *reinterpret_cast<uint32_t(*)[16]>(&sr[16]));
                 tmem_wait_ld();
                 tc_fence_before();
                 __syncwarp();
@@ -636,17 +583,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
                 uint32_t pak[WITH_RHO ? GCOLS / 2 : 1];
                 if constexpr (WITH_RHO) {
-                    // ---- A of this group's 32 keys, then release X ----
+                    // ---- A of this group's 32 keys (its P goes over them) ----
                     if (!warp_wait(smem_u32(&bars->a_full), G & 1, wc)) { ok = false; break; }
                     tc_fence_after();
                     uint32_t ar[GCOLS];
-                    tmem_ld16(tmem + lane_off + COL_X + grp * GCOLS, *reinterpret_cast<uint32_t(*)[16]>(&ar[0]));
-                    tmem_ld16(tmem + lane_off + COL_X + grp * GCOLS + 16,
-                              *reinterpret_cast<uint32_t(*)[16]>(&ar[16]));
+                    tmem_ld16(xcol, *reinterpret_cast<uint32_t(*)[16]>(&ar[0]));
+                    tmem_ld16(xcol + 16, *reinterpret_cast<uint32_t(*)[16]>(&ar[16]));
                     tmem_wait_ld();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(smem_u32(&bars->a_free));
                     float a4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int i = 0; i < GCOLS / 2; ++i) {
@@ -656,12 +599,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         a4[i & 3] = add_f16x2_to_f32(a4[i & 3], pak[i]);
                     }
                     ab += (a4[0] + a4[1]) + (a4[2] + a4[3]);
-                }
-                // ---- the previous tile's P.V UMMAs are done: the P region is
-                // free and O, M' hold every earlier tile of this item ----
-                if (G > 0) {
-                    if (!warp_wait(smem_u32(&bars->pv_done), (G - 1) & 1, wc)) { ok = false; break; }
-                    tc_fence_after();
                 }
                 // ---- V of this block holds v 2^-e: P and P o A' are stored as
                 // 2^e P and 2^e P o A', so the P.V products are unchanged (a
@@ -679,7 +616,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     }
                 }
                 // a moved reference max rescales O and M' (each group d/4 columns)
+                // once the previous tile's P.V UMMAs are done: O and M' then hold
+                // every earlier tile of this item, and this tile's are not issued
                 if (__any_sync(0xffffffffu, moved && j > 0)) {
+                    if (!warp_wait(smem_u32(&bars->pv_done[(G - 1) & 1]), ((G - 1) >> 1) & 1, wc)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
                     const float f = (moved && j > 0) ? alpha : 1.f;
 #pragma unroll 1
                     for (int c = grp * Gm::OCOLS; c < grp * Gm::OCOLS + Gm::OCOLS; c += 16) {
@@ -698,13 +642,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         }
                     }
                 }
-                // ---- P and P o A' into this group's P columns, for the P.V UMMAs ----
-                tmem_st16(tmem + lane_off + COL_P + grp * GCOLS, pk);
-                if constexpr (WITH_RHO) tmem_st16(tmem + lane_off + COL_P + grp * GCOLS + PA_SHIFT, pak);
+                // ---- P and P o A' over this group's S and A columns, for the P.V UMMAs ----
+                tmem_st16(xcol, pk);
+                if constexpr (WITH_RHO) tmem_st16(xcol + PA_SHIFT, pak);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&bars->p_full));
+                if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[G & 1]));
             }
             if (!ok) break;
             // ---------------------------------------------- epilogue --
@@ -719,7 +663,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const float abt = (bars->red_sum[1][0][r] + bars->red_sum[1][1][r]) +
                               (bars->red_sum[1][2][r] + bars->red_sum[1][3][r]);
             // the last P.V UMMAs of this item are done: O and M' are final
-            if (!warp_wait(smem_u32(&bars->pv_done), (G - 1) & 1, wc)) break;
+            if (!warp_wait(smem_u32(&bars->pv_done[(G - 1) & 1]), ((G - 1) >> 1) & 1, wc)) break;
             tc_fence_after();
             const float inv_l = 1.0f / lt;
             const float abar = abt * inv_l;

@@ -1,6 +1,6 @@
 """Derivation of the polynomial 2^x the prefill kernel uses for part of its exponentials.
 
-The kernel (``csrc/fwd_sm100.cu``, ``exp2_poly2``) reduces 2^x = 2^j * 2^f with
+The prefill kernels (``csrc/softmax_sm100.cuh``, ``exp2_poly2``) reduce 2^x = 2^j * 2^f with
 j = round(x) and f = x - j in [-1/2, 1/2], and evaluates 2^f with a degree-3
 polynomial.  The coefficients are the minimax fit of 2^f on [-1/2, 1/2] in
 relative error, found here with the Remez exchange algorithm (alternation of
@@ -13,7 +13,7 @@ import re
 
 import numpy as np
 
-_CU = os.path.join(os.path.dirname(os.path.abspath(__file__)), "csrc", "fwd_sm100.cu")
+_CU = os.path.join(os.path.dirname(os.path.abspath(__file__)), "csrc", "softmax_sm100.cuh")
 
 
 def remez_exp2(degree=3, lo=-0.5, hi=0.5, iters=40, grid=200001):
