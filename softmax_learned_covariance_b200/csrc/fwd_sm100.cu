@@ -161,6 +161,26 @@ __device__ __forceinline__ Item item_of(int w, int BH, int nq, int T, int causal
     return it;
 }
 
+// P = exp2(s log2e/sqrt(d) - m_ref) for N key pairs, rounded to fp16 pairs;
+// three pairs in eight go through the FMA-pipe polynomial.
+template <int N>
+__device__ __forceinline__ void weights_f16(const uint32_t (&sr)[2 * N], uint32_t (&pk)[N], float scale_log2,
+                                            float neg_m) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        float x0, x1;
+        ffma2(x0, x1, __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]), scale_log2, neg_m);
+        float e0, e1;
+        if ((i & 7) == 1 || (i & 7) == 4 || (i & 7) == 7) {
+            exp2_poly2(e0, e1, x0, x1);
+        } else {
+            e0 = ex2(x0);
+            e1 = ex2(x1);
+        }
+        pk[i] = pack_f16x2(e0, e1);
+    }
+}
+
 template <int D, bool WITH_RHO, bool FUSED, typename Tout>
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -469,6 +489,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int r = quarter * 32 + lane;               // query row within the tile == TMEM lane
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const float scale_log2 = LOG2E / sqrtf((float)D);
+        // 32-byte output stores (half the store instructions of 16-byte ones)
+        // when the output rows are 32-byte aligned; the same for every thread
+        const bool wide = ((reinterpret_cast<uintptr_t>(y) | reinterpret_cast<uintptr_t>(o_out)) & 31) == 0;
         const int vsg = (grp * GCOLS) / VKEYS;           // the V block (within a tile) of this group's keys
         const int nblk = (T + VKEYS - 1) / VKEYS;        // 64-key V blocks per head, one exponent each
         uint32_t G = 0, ni = 0;   // key tiles and items processed by this CTA
@@ -549,38 +572,55 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 bars->red_max[G & 1][grp][r] = mx;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&bars->xchg[G & 1]));
-                if (!warp_wait(smem_u32(&bars->xchg[G & 1]), (G >> 1) & 1, wc)) { ok = false; break; }
-                mx = fmaxf(fmaxf(bars->red_max[G & 1][0][r], bars->red_max[G & 1][1][r]),
-                           fmaxf(bars->red_max[G & 1][2][r], bars->red_max[G & 1][3][r])) *
-                     scale_log2;
                 float alpha = 1.f;
                 bool moved = false;
-                if (mx > m_ref + RESCALE_THRESHOLD) {
-                    alpha = ex2(m_ref - mx);     // 0 when m_ref = -inf
-                    m_ref = mx;
-                    l *= alpha;
-                    ab *= alpha;
-                    moved = true;
-                }
-                // ---- P = exp2(z log2e - m_ref) as fp16, sums from the rounded values ----
-                const float neg_m = -m_ref;
                 uint32_t pk[GCOLS / 2];
-                float l4[4] = {0.f, 0.f, 0.f, 0.f};
+                // ---- P = exp2(z log2e - m_ref) as fp16.  While the other groups'
+                // maxima arrive, P is formed with the current reference when no
+                // score of this warp's own keys needs it moved (after an item's
+                // first tile, nearly always); if another group's keys move it, the
+                // fp16 P is scaled to the new reference (weights below 2^8, so no
+                // overflow).  Otherwise P waits for the row max as usual. ----
+                const bool spec =
+                    __all_sync(0xffffffffu, m_ref != -INFINITY && mx * scale_log2 <= m_ref + RESCALE_THRESHOLD);
+                if (spec) {
+                    weights_f16(sr, pk, scale_log2, -m_ref);
+                    if (!warp_wait(smem_u32(&bars->xchg[G & 1]), (G >> 1) & 1, wc)) { ok = false; break; }
+                    mx = fmaxf(fmaxf(bars->red_max[G & 1][0][r], bars->red_max[G & 1][1][r]),
+                               fmaxf(bars->red_max[G & 1][2][r], bars->red_max[G & 1][3][r])) *
+                         scale_log2;
+                    if (mx > m_ref + RESCALE_THRESHOLD) {
+                        alpha = ex2(m_ref - mx);
+                        m_ref = mx;
+                        l *= alpha;
+                        ab *= alpha;
+                        moved = true;
+                        const __half2 f2 = __float2half2_rn(alpha);
+                        const uint32_t fh = *reinterpret_cast<const uint32_t *>(&f2);
 #pragma unroll
-                for (int i = 0; i < GCOLS / 2; ++i) {
-                    float x0, x1;
-                    ffma2(x0, x1, __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]), scale_log2, neg_m);
-                    float e0, e1;
-                    if ((i & 7) == 1 || (i & 7) == 4 || (i & 7) == 7) {
-                        exp2_poly2(e0, e1, x0, x1);   // three pairs in eight on the FMA pipe
-                    } else {
-                        e0 = ex2(x0);
-                        e1 = ex2(x1);
+                        for (int i = 0; i < GCOLS / 2; ++i) pk[i] = hmul2(pk[i], fh);
                     }
-                    pk[i] = pack_f16x2(e0, e1);
-                    l4[i & 3] = add_f16x2_to_f32(l4[i & 3], pk[i]);
+                } else {
+                    if (!warp_wait(smem_u32(&bars->xchg[G & 1]), (G >> 1) & 1, wc)) { ok = false; break; }
+                    mx = fmaxf(fmaxf(bars->red_max[G & 1][0][r], bars->red_max[G & 1][1][r]),
+                               fmaxf(bars->red_max[G & 1][2][r], bars->red_max[G & 1][3][r])) *
+                         scale_log2;
+                    if (mx > m_ref + RESCALE_THRESHOLD) {
+                        alpha = ex2(m_ref - mx);     // 0 when m_ref = -inf
+                        m_ref = mx;
+                        l *= alpha;
+                        ab *= alpha;
+                        moved = true;
+                    }
+                    weights_f16(sr, pk, scale_log2, -m_ref);
                 }
-                l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+                // ---- row sums from the rounded weights the MMAs read ----
+                {
+                    float l4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int i = 0; i < GCOLS / 2; ++i) l4[i & 3] = add_f16x2_to_f32(l4[i & 3], pk[i]);
+                    l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+                }
                 uint32_t pak[WITH_RHO ? GCOLS / 2 : 1];
                 if constexpr (WITH_RHO) {
                     // ---- A of this group's 32 keys (its P goes over them) ----
@@ -689,19 +729,35 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     finite = finite && isfinite(out[i]);
                 }
                 if (store && o_out != nullptr) {   // training forward: o = O / l for the backward
-                    float4 *dst = reinterpret_cast<float4 *>(o_out + ((size_t)it.bh * T + qrow) * D + c);
+                    float *dst = o_out + ((size_t)it.bh * T + qrow) * D + c;
+                    if (wide) {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv_l, __uint_as_float(o[4 * i + 1]) * inv_l,
-                                             __uint_as_float(o[4 * i + 2]) * inv_l,
-                                             __uint_as_float(o[4 * i + 3]) * inv_l);
+                        for (int h = 0; h < 2; ++h) {
+                            uint32_t w8[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) w8[i] = __float_as_uint(__uint_as_float(o[8 * h + i]) * inv_l);
+                            st_global_v8(dst + 8 * h, w8);
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            reinterpret_cast<float4 *>(dst)[i] =
+                                make_float4(__uint_as_float(o[4 * i]) * inv_l, __uint_as_float(o[4 * i + 1]) * inv_l,
+                                            __uint_as_float(o[4 * i + 2]) * inv_l, __uint_as_float(o[4 * i + 3]) * inv_l);
+                    }
                 }
                 if (store) {
                     if constexpr (sizeof(Tout) == 4) {
-                        float4 *dst = reinterpret_cast<float4 *>(yrow + c);
+                        if (wide) {
 #pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            dst[i] = make_float4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
+                            for (int h = 0; h < 2; ++h)
+                                st_global_v8(yrow + c + 8 * h, *reinterpret_cast<const uint32_t(*)[8]>(&out[8 * h]));
+                        } else {
+                            float4 *dst = reinterpret_cast<float4 *>(yrow + c);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                dst[i] = make_float4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
+                        }
                     } else {
                         uint32_t pb[8];
 #pragma unroll
@@ -709,9 +765,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                             __nv_bfloat162 h = __floats2bfloat162_rn(out[2 * i], out[2 * i + 1]);
                             pb[i] = *reinterpret_cast<uint32_t *>(&h);
                         }
-                        uint4 *dst = reinterpret_cast<uint4 *>(yrow + c);
-                        dst[0] = make_uint4(pb[0], pb[1], pb[2], pb[3]);
-                        dst[1] = make_uint4(pb[4], pb[5], pb[6], pb[7]);
+                        if (wide) {
+                            st_global_v8(yrow + c, pb);
+                        } else {
+                            uint4 *dst = reinterpret_cast<uint4 *>(yrow + c);
+                            dst[0] = make_uint4(pb[0], pb[1], pb[2], pb[3]);
+                            dst[1] = make_uint4(pb[4], pb[5], pb[6], pb[7]);
+                        }
                     }
                 }
             }
