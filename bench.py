@@ -80,11 +80,11 @@ def decode_bytes(B, H, d, seqlens):
 
 
 # DRAM bytes per algorithmic byte of the decode kernel, from an ncu capture of
-# the same kernel at B=16 H=16 ctx 8192 (1.0739 GB read + 0.0078 GB written for
+# the same kernel at B=16 H=16 ctx 8192 (1.0739 GB read + 0.0099 GB written for
 # 1.0740 GB of K/V rows, q, rho and y).  Traffic grows in proportion to the
 # cached tokens read, so a launch's traffic is this ratio times its algorithmic
 # bytes.
-DECODE_TRAFFIC_RATIO = 1.0818 / 1.0740
+DECODE_TRAFFIC_RATIO = 1.0838 / 1.0740
 
 
 def prefill_pairs(B, H, T, causal=True):
