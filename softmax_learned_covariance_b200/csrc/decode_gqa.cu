@@ -18,14 +18,20 @@
 //
 // With one query head per KV head the operand is mostly zero rows, but the
 // per-warp cp.async ring still hides the page indirection better than the
-// per-head CUDA-core decode did (B=64 ctx 4096: 0.83 against 0.68 of HBM).
+// per-head CUDA-core decode did (B=64 ctx 4096: 0.92 against 0.68 of HBM).
 //
 // A CTA of 4 warps takes one (sequence, KV head, up to 8 query heads, chunk)
 // unit; each warp streams its own 16-token tiles of the chunk through a
-// 3-stage cp.async ring in shared memory (128-byte-row swizzle, read back with
+// 2-stage cp.async ring in shared memory (128-byte-row swizzle, read back with
 // ldmatrix) and keeps its own online-softmax state; the four states are
 // merged at the end and written as the same partials (or y) as the split
 // kernel, so the split combine applies unchanged.
+//
+// Occupancy over depth (measured, B=64 Hq=32 Hkv=8 ctx 4096): a 3-stage ring
+// at 2 CTAs per SM (210 registers, 96 KB each) streamed 0.73 of HBM; a
+// 2-stage ring at 3 CTAs per SM (registers capped at 170, no spills) 0.84,
+// and 0.92 with one query head per KV head; 4 CTAs per SM (128 registers)
+// spilled and fell to 0.69.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <math.h>
@@ -37,7 +43,8 @@ namespace {
 
 constexpr int WARPS = 4;
 constexpr int TILE = 16;      // tokens per warp step
-constexpr int STAGES = 3;    // tiles in flight per warp: STAGES - 1
+constexpr int STAGES = 2;    // tiles in flight per warp: STAGES - 1
+constexpr int MIN_CTAS = 3;  // resident CTAs per SM (registers capped at 170, 64 KB of ring each)
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 
@@ -118,7 +125,7 @@ template <int D> struct GqaSmem {
 };
 
 template <int D, typename Tout>
-__global__ void __launch_bounds__(WARPS * 32) k_decode_gqa(
+__global__ void __launch_bounds__(WARPS * 32, MIN_CTAS) k_decode_gqa(
     const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ rho, const __nv_bfloat16 *__restrict__ kp,
     const __nv_bfloat16 *__restrict__ vp, const int *__restrict__ seqlens, Tout *__restrict__ y,
     float *__restrict__ lse, int Hq, int chunk, int nsplit, long units_per_split, int htiles, PagedKV pg,
