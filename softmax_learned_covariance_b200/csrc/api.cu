@@ -297,13 +297,24 @@ int parallax_bwd(const void *q, const void *k, const void *v, const void *rho, c
     int st = get_state(&s);
     if (st) return st;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    // scratch: go and delta per row
+    if ((st = ensure_encoder())) return st;
+    // scratch: the dq kernel's work counter, then go and delta per row
     CallScratch scratch(s, cs);
     void *ws = nullptr;
     const size_t rows = (size_t)B * H * T;
-    if ((st = scratch.get(2 * rows * sizeof(float), &ws))) return st;
-    float *go = static_cast<float *>(ws), *delta = go + rows;
-    return status_of(launch_bwd(q, k, v, rho, dy, y, o, abar, lse, go, delta, dq, dk, dv, drho, B, H, T, d, causal, cs));
+    if ((st = scratch.get(256 + 2 * rows * sizeof(float), &ws))) return st;
+    int *counter = static_cast<int *>(ws);
+    float *go = reinterpret_cast<float *>(static_cast<char *>(ws) + 256), *delta = go + rows;
+    BwdTensorMaps tm;
+    const uint64_t dims[3] = {(uint64_t)d, (uint64_t)T, (uint64_t)B * H};
+    const uint32_t box[3] = {64, 128, 1};
+    if ((st = encode(&tm.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, 3, dims, box, 2))) return st;
+    if ((st = encode(&tm.r, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rho, 3, dims, box, 2))) return st;
+    if ((st = encode(&tm.g, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dy, 3, dims, box, 2))) return st;
+    if ((st = encode(&tm.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k, 3, dims, box, 2))) return st;
+    if ((st = encode(&tm.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v, 3, dims, box, 2))) return st;
+    return status_of(launch_bwd(q, k, v, rho, dy, y, o, abar, lse, go, delta, dq, dk, dv, drho, B, H, T, d, causal, tm,
+                                s->sms, counter, make_ctl(s), cs));
 }
 
 int parallax_fwd_fused(const void *q, const void *k, const void *v, const void *x, const void *W_R, void *y,

@@ -14,16 +14,16 @@
 //                                                          dk_j  += sum_i dA_ij rho_i)
 // lse_i, abar_i and o_i come from the training forward (parallax_fwd_train).
 //
-// Three kernels: k_bwd_rowstats (go, delta per row), k_bwd_dq (query blocks of
-// 64 rows, looping over the keys: dq and drho accumulate in registers) and
-// k_bwd_dkdv (key blocks of 64, looping over the queries: dk and dv accumulate
-// in registers).  Both main kernels recompute S, A and G from q, k, rho, v and
-// dY, so no gradient needs atomics and the result is deterministic.  The
-// products run on warp-level mma.sync (m16n8k16, bf16 operands, fp32
+// Three kernels: k_bwd_rowstats (go, delta per row), the tensor-core dq / drho
+// kernel of bwd_sm100.cu (query tiles of 128 rows, looping over the keys) and
+// k_bwd_dkdv here (key blocks of 64, looping over the queries: dk and dv
+// accumulate in registers).  Both main kernels recompute S, A and G from q, k,
+// rho, v and dY, so no gradient needs atomics and the result is deterministic.
+// k_bwd_dkdv runs on warp-level mma.sync (m16n8k16, bf16 operands, fp32
 // accumulation): W, dZ and dA are rounded to bf16 as operands (relative error
-// 2^-9 per weight).  Operand tiles are staged in shared memory with 16-byte
-// chunks XOR-swizzled by row, loaded with cp.async (double-buffered) and read
-// with ldmatrix.
+// 2^-9 per weight), as in the dq kernel.  Operand tiles are staged in shared
+// memory with 16-byte chunks XOR-swizzled by row, loaded with cp.async
+// (double-buffered) and read with ldmatrix.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -131,131 +131,6 @@ __global__ void __launch_bounds__(256) k_bwd_rowstats(const __nv_bfloat16 *__res
     if (lane == 0) {
         go[row] = so;
         delta[row] = sy + abar[row] * so;
-    }
-}
-
-// ------------------------------------------------- dq, drho per query block --
-template <int D>
-__global__ void __launch_bounds__(NT, 2)
-    k_bwd_dq(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-             const __nv_bfloat16 *__restrict__ v, const __nv_bfloat16 *__restrict__ rho,
-             const __nv_bfloat16 *__restrict__ dy, const float *__restrict__ lse, const float *__restrict__ abar,
-             const float *__restrict__ go, const float *__restrict__ delta, float *__restrict__ dq,
-             float *__restrict__ drho, int T, int causal) {
-    constexpr int ROWB = BR * D * 2, COLB = BC * D * 2, ND = D / 8;
-    extern __shared__ __align__(128) uint8_t sm[];
-    const uint32_t sQ = (uint32_t)__cvta_generic_to_shared(sm), sR = sQ + ROWB, sG = sR + ROWB;
-    const uint32_t sK0 = sG + ROWB;   // K[buf] at sK0 + buf * 2 * COLB, V[buf] just after
-    const int warp = threadIdx.x / 32, lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
-    const long bh = blockIdx.y;
-    const int row0 = blockIdx.x * BR;
-    const size_t hb = (size_t)bh * T;
-    const float sc = LOG2E / sqrtf((float)D), inv_sqrt = 1.0f / sqrtf((float)D);
-
-    load_tile<D>(sQ, q + (hb + row0) * D, BR, T - row0);
-    load_tile<D>(sR, rho + (hb + row0) * D, BR, T - row0);
-    load_tile<D>(sG, dy + (hb + row0) * D, BR, T - row0);
-    const int kend = causal ? min(T, row0 + BR) : T;
-    const int nsteps = (kend + BC - 1) / BC;
-    auto load_cols = [&](int st) {
-        const uint32_t b = sK0 + (st & 1) * 2 * COLB;
-        load_tile<D>(b, k + (hb + (size_t)st * BC) * D, BC, T - st * BC);
-        load_tile<D>(b + COLB, v + (hb + (size_t)st * BC) * D, BC, T - st * BC);
-    };
-    load_cols(0);
-    cp_async_commit();
-
-    // statistics of this thread's two rows
-    int rr[2] = {row0 + 16 * warp + gq, row0 + 16 * warp + gq + 8};
-    float l2[2], ab[2], gov[2], dl[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const bool ok = rr[h] < T;
-        l2[h] = ok ? lse[hb + rr[h]] * LOG2E : INFINITY;   // rows past T get zero weights
-        ab[h] = ok ? abar[hb + rr[h]] : 0.f;
-        gov[h] = ok ? go[hb + rr[h]] : 0.f;
-        dl[h] = ok ? delta[hb + rr[h]] : 0.f;
-    }
-    float aq[ND][4], ar[ND][4];
-#pragma unroll
-    for (int t = 0; t < ND; ++t)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) aq[t][e] = ar[t][e] = 0.f;
-
-    for (int st = 0; st < nsteps; ++st) {
-        if (st + 1 < nsteps) load_cols(st + 1);
-        cp_async_commit();
-        cp_async_wait<1>();
-        __syncthreads();
-        const uint32_t sK = sK0 + (st & 1) * 2 * COLB, sV = sK + COLB;
-        // S = Q K^T, A = R K^T, G = dY V^T for 16 rows x 32 keys
-        float s4[4][4], a4[4][4], g4[4][4];
-#pragma unroll
-        for (int t = 0; t < 4; ++t)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) s4[t][e] = a4[t][e] = g4[t][e] = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-            uint32_t fq[4], fr[4], fg[4];
-            lda<D>(sQ, 16 * warp, kk, fq);
-            lda<D>(sR, 16 * warp, kk, fr);
-            lda<D>(sG, 16 * warp, kk, fg);
-#pragma unroll
-            for (int nb = 0; nb < 2; ++nb) {
-                uint32_t bk[4], bv[4];
-                ldb<D>(sK, 16 * nb, kk, bk);
-                ldb<D>(sV, 16 * nb, kk, bv);
-                mma16816(s4[2 * nb], fq, bk[0], bk[1]);
-                mma16816(s4[2 * nb + 1], fq, bk[2], bk[3]);
-                mma16816(a4[2 * nb], fr, bk[0], bk[1]);
-                mma16816(a4[2 * nb + 1], fr, bk[2], bk[3]);
-                mma16816(g4[2 * nb], fg, bv[0], bv[1]);
-                mma16816(g4[2 * nb + 1], fg, bv[2], bv[3]);
-            }
-        }
-        // dZ / sqrt(d) and dA as bf16 A fragments, k = the 32 keys in two steps of 16
-        uint32_t fz[2][4], fa[2][4];
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-            float z[4], a[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int h = e >> 1;
-                const int key = st * BC + 8 * t + 2 * tq + (e & 1);
-                const bool ok = key < T && (!causal || key <= rr[h]);
-                const float s = ok ? exp2f(fmaf(s4[t][e], sc, -l2[h])) : 0.f;
-                const float av = a4[t][e], gv = g4[t][e];
-                z[e] = s * (fmaf(1.f + ab[h] - av, gv, av * gov[h]) - dl[h]) * inv_sqrt;
-                a[e] = s * (gov[h] - gv);
-            }
-            fz[t >> 1][(t & 1) * 2 + 0] = pack_bf16(z[0], z[1]);
-            fz[t >> 1][(t & 1) * 2 + 1] = pack_bf16(z[2], z[3]);
-            fa[t >> 1][(t & 1) * 2 + 0] = pack_bf16(a[0], a[1]);
-            fa[t >> 1][(t & 1) * 2 + 1] = pack_bf16(a[2], a[3]);
-        }
-        // dq += dZ K / sqrt(d), drho += dA K
-#pragma unroll
-        for (int m = 0; m < 2; ++m)
-#pragma unroll
-            for (int nd = 0; nd < D / 16; ++nd) {
-                uint32_t b[4];
-                ldb_t<D>(sK, m, nd, b);
-                mma16816(aq[2 * nd], fz[m], b[0], b[1]);
-                mma16816(aq[2 * nd + 1], fz[m], b[2], b[3]);
-                mma16816(ar[2 * nd], fa[m], b[0], b[1]);
-                mma16816(ar[2 * nd + 1], fa[m], b[2], b[3]);
-            }
-        __syncthreads();   // this buffer is refilled two steps on
-    }
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        if (rr[h] >= T) continue;
-        float *pq = dq + (hb + rr[h]) * D, *pr = drho + (hb + rr[h]) * D;
-#pragma unroll
-        for (int t = 0; t < ND; ++t) {
-            *reinterpret_cast<float2 *>(pq + 8 * t + 2 * tq) = make_float2(aq[t][2 * h], aq[t][2 * h + 1]);
-            *reinterpret_cast<float2 *>(pr + 8 * t + 2 * tq) = make_float2(ar[t][2 * h], ar[t][2 * h + 1]);
-        }
     }
 }
 
@@ -398,22 +273,22 @@ __global__ void __launch_bounds__(NT, 2)
 template <int D>
 cudaError_t launch_t(const void *q, const void *k, const void *v, const void *rho, const void *dy, const float *y,
                      const float *o, const float *abar, const float *lse, float *go, float *delta, float *dq,
-                     float *dk, float *dv, float *drho, int BH, int T, int causal, cudaStream_t s) {
+                     float *dk, float *dv, float *drho, int B, int H, int T, int causal, const BwdTensorMaps &tm,
+                     int sm_count, int *work_counter, const DeviceCtl &ctl, cudaStream_t s) {
+    const int BH = B * H;
     using bf = __nv_bfloat16;
     const long rows = (long)BH * T;
     k_bwd_rowstats<D><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>((const bf *)dy, o, y, abar, go, delta, rows);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     constexpr int ROWB = BR * D * 2, COLB = BC * D * 2;
-    constexpr int SM_DQ = 3 * ROWB + 4 * COLB;
     constexpr int SM_DK = 2 * ROWB + 2 * (3 * COLB + 4 * BC * 4);
-    static std::atomic<unsigned long long> set_dq{0}, set_dk{0};
-    if ((e = ensure_smem_limit(k_bwd_dq<D>, SM_DQ, set_dq))) return e;
+    static std::atomic<unsigned long long> set_dk{0};
     if ((e = ensure_smem_limit(k_bwd_dkdv<D>, SM_DK, set_dk))) return e;
     const dim3 grid((unsigned)((T + BR - 1) / BR), (unsigned)BH);
-    k_bwd_dq<D><<<grid, NT, SM_DQ, s>>>((const bf *)q, (const bf *)k, (const bf *)v, (const bf *)rho, (const bf *)dy,
-                                       lse, abar, go, delta, dq, drho, T, causal);
-    if ((e = cudaGetLastError())) return e;
+    if ((e = launch_bwd_dq_sm100(tm, lse, abar, go, delta, dq, drho, B, H, T, D, causal, sm_count, work_counter, ctl,
+                                 s)))
+        return e;
     k_bwd_dkdv<D><<<grid, NT, SM_DK, s>>>((const bf *)q, (const bf *)k, (const bf *)v, (const bf *)rho,
                                          (const bf *)dy, lse, abar, go, delta, dk, dv, T, causal);
     return cudaGetLastError();
@@ -423,10 +298,13 @@ cudaError_t launch_t(const void *q, const void *k, const void *v, const void *rh
 
 cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *rho, const void *dy, const float *y,
                        const float *o, const float *abar, const float *lse, float *go, float *delta, float *dq,
-                       float *dk, float *dv, float *drho, int B, int H, int T, int d, int causal, cudaStream_t s) {
+                       float *dk, float *dv, float *drho, int B, int H, int T, int d, int causal,
+                       const BwdTensorMaps &tm, int sm_count, int *work_counter, const DeviceCtl &ctl, cudaStream_t s) {
     if (d == 64)
-        return launch_t<64>(q, k, v, rho, dy, y, o, abar, lse, go, delta, dq, dk, dv, drho, B * H, T, causal, s);
-    return launch_t<128>(q, k, v, rho, dy, y, o, abar, lse, go, delta, dq, dk, dv, drho, B * H, T, causal, s);
+        return launch_t<64>(q, k, v, rho, dy, y, o, abar, lse, go, delta, dq, dk, dv, drho, B, H, T, causal, tm, sm_count,
+                            work_counter, ctl, s);
+    return launch_t<128>(q, k, v, rho, dy, y, o, abar, lse, go, delta, dq, dk, dv, drho, B, H, T, causal, tm, sm_count,
+                         work_counter, ctl, s);
 }
 
 }  // namespace plx

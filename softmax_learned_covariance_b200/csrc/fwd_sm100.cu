@@ -161,26 +161,6 @@ __device__ __forceinline__ Item item_of(int w, int BH, int nq, int T, int causal
     return it;
 }
 
-// P = exp2(s log2e/sqrt(d) - m_ref) for N key pairs, rounded to fp16 pairs;
-// three pairs in eight go through the FMA-pipe polynomial.
-template <int N>
-__device__ __forceinline__ void weights_f16(const uint32_t (&sr)[2 * N], uint32_t (&pk)[N], float scale_log2,
-                                            float neg_m) {
-#pragma unroll
-    for (int i = 0; i < N; ++i) {
-        float x0, x1;
-        ffma2(x0, x1, __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]), scale_log2, neg_m);
-        float e0, e1;
-        if ((i & 7) == 1 || (i & 7) == 4 || (i & 7) == 7) {
-            exp2_poly2(e0, e1, x0, x1);
-        } else {
-            e0 = ex2(x0);
-            e1 = ex2(x1);
-        }
-        pk[i] = pack_f16x2(e0, e1);
-    }
-}
-
 template <int D, bool WITH_RHO, bool FUSED, typename Tout>
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,

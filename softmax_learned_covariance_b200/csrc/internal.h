@@ -102,11 +102,23 @@ cudaError_t launch_fwd_fused_sm100(const FwdTensorMaps &tm, void *y, float *lse,
                                    int H, int T, int d_model, int causal, int out_dtype, int sm_count,
                                    int *work_counter, const DeviceCtl &ctl, cudaStream_t s);
 
+// Tensor maps of the tensor-core dq / drho kernel: q, rho, dY, k and v, each
+// [B*H rows of T x d] bf16 seen as {d, T, B*H}, 128-byte swizzled boxes of
+// 64 columns x 128 rows.
+struct BwdTensorMaps {
+    CUtensorMap q, r, g, k, v;
+};
+// dq and drho (fp32, [B,H,T,d]) from lse, abar (training forward) and go, delta
+// (k_bwd_rowstats) on tcgen05 (bwd_sm100.cu); work_counter: one int of scratch.
+cudaError_t launch_bwd_dq_sm100(const BwdTensorMaps &tm, const float *lse, const float *abar, const float *go,
+                                const float *delta, float *dq, float *drho, int B, int H, int T, int d, int causal,
+                                int sm_count, int *work_counter, const DeviceCtl &ctl, cudaStream_t s);
 // Gradients of the prefill (mma.sync kernels): go, delta are [B*H*T] fp32
 // scratch; q, k, v, rho, dy bf16; y, o fp32 [B,H,T,d]; abar, lse fp32 [B,H,T];
 // dq, dk, dv, drho fp32 [B,H,T,d] (written).
 cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *rho, const void *dy, const float *y,
                        const float *o, const float *abar, const float *lse, float *go, float *delta, float *dq,
-                       float *dk, float *dv, float *drho, int B, int H, int T, int d, int causal, cudaStream_t s);
+                       float *dk, float *dv, float *drho, int B, int H, int T, int d, int causal, const BwdTensorMaps &tm,
+                       int sm_count, int *work_counter, const DeviceCtl &ctl, cudaStream_t s);
 
 }  // namespace plx

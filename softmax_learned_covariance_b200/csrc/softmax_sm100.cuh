@@ -78,6 +78,27 @@ __device__ __forceinline__ void exp2_poly2(float &y0, float &y1, float x0, float
     y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
+// exp2(s c - m) for N pairs of fp32 values s, rounded to fp16 pairs (the
+// softmax weights P of the prefill, s of the backward); three pairs in eight
+// go through the FMA-pipe polynomial.
+template <int N>
+__device__ __forceinline__ void weights_f16(const uint32_t (&sr)[2 * N], uint32_t (&pk)[N], float scale_log2,
+                                            float neg_m) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        float x0, x1;
+        ffma2(x0, x1, __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]), scale_log2, neg_m);
+        float e0, e1;
+        if ((i & 7) == 1 || (i & 7) == 4 || (i & 7) == 7) {
+            exp2_poly2(e0, e1, x0, x1);
+        } else {
+            e0 = ex2(x0);
+            e1 = ex2(x1);
+        }
+        pk[i] = pack_f16x2(e0, e1);
+    }
+}
+
 // One 32-byte global store (8 words); the address must be 32-byte aligned.
 __device__ __forceinline__ void st_global_v8(void *p, const uint32_t (&w)[8]) {
     asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]),
