@@ -298,23 +298,28 @@ int parallax_bwd(const void *q, const void *k, const void *v, const void *rho, c
     if (st) return st;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     if ((st = ensure_encoder())) return st;
-    // scratch: the dq kernel's work counter, then go and delta per row
+    // scratch: the two gradient kernels' work counters, go and delta per row,
+    // then the packed per-query statistics (rows padded to a multiple of 64 per head)
     CallScratch scratch(s, cs);
     void *ws = nullptr;
-    const size_t rows = (size_t)B * H * T;
-    if ((st = scratch.get(256 + 2 * rows * sizeof(float), &ws))) return st;
-    int *counter = static_cast<int *>(ws);
+    const size_t rows = (size_t)B * H * T, prows = (size_t)B * H * bwd_tpad(T);
+    const size_t off_st = (256 + 2 * rows * sizeof(float) + 255) & ~(size_t)255;
+    if ((st = scratch.get(off_st + prows * 16, &ws))) return st;
+    int *counters = static_cast<int *>(ws);
     float *go = reinterpret_cast<float *>(static_cast<char *>(ws) + 256), *delta = go + rows;
-    BwdTensorMaps tm;
+    void *st4 = static_cast<char *>(ws) + off_st;
+    BwdTensorMaps tq, tk;
     const uint64_t dims[3] = {(uint64_t)d, (uint64_t)T, (uint64_t)B * H};
-    const uint32_t box[3] = {64, 128, 1};
-    if ((st = encode(&tm.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, 3, dims, box, 2))) return st;
-    if ((st = encode(&tm.r, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rho, 3, dims, box, 2))) return st;
-    if ((st = encode(&tm.g, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dy, 3, dims, box, 2))) return st;
-    if ((st = encode(&tm.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k, 3, dims, box, 2))) return st;
-    if ((st = encode(&tm.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v, 3, dims, box, 2))) return st;
-    return status_of(launch_bwd(q, k, v, rho, dy, y, o, abar, lse, go, delta, dq, dk, dv, drho, B, H, T, d, causal, tm,
-                                s->sms, counter, make_ctl(s), cs));
+    const uint32_t box128[3] = {64, 128, 1}, box64[3] = {64, 64, 1};
+    const void *src[5] = {q, rho, dy, k, v};
+    CUtensorMap *mq[5] = {&tq.q, &tq.r, &tq.g, &tq.k, &tq.v}, *mk[5] = {&tk.q, &tk.r, &tk.g, &tk.k, &tk.v};
+    for (int i = 0; i < 5; ++i) {
+        if ((st = encode(mq[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, src[i], 3, dims, box128, 2))) return st;
+        if ((st = encode(mk[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, src[i], 3, dims, i < 3 ? box64 : box128, 2)))
+            return st;
+    }
+    return status_of(launch_bwd(dy, y, o, abar, lse, go, delta, st4, dq, dk, dv, drho, B, H, T, d, causal, tq, tk,
+                                s->sms, counters, make_ctl(s), cs));
 }
 
 int parallax_fwd_fused(const void *q, const void *k, const void *v, const void *x, const void *W_R, void *y,

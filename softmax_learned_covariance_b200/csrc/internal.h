@@ -102,9 +102,10 @@ cudaError_t launch_fwd_fused_sm100(const FwdTensorMaps &tm, void *y, float *lse,
                                    int H, int T, int d_model, int causal, int out_dtype, int sm_count,
                                    int *work_counter, const DeviceCtl &ctl, cudaStream_t s);
 
-// Tensor maps of the tensor-core dq / drho kernel: q, rho, dY, k and v, each
-// [B*H rows of T x d] bf16 seen as {d, T, B*H}, 128-byte swizzled boxes of
-// 64 columns x 128 rows.
+// Tensor maps of the tensor-core gradient kernels: q, rho, dY, k and v, each
+// [B*H rows of T x d] bf16 seen as {d, T, B*H}, 128-byte swizzled boxes of 64
+// columns x 128 rows (the dq / drho kernel) or x 64 rows for q, rho, dY (the
+// dk / dv kernel).
 struct BwdTensorMaps {
     CUtensorMap q, r, g, k, v;
 };
@@ -113,12 +114,20 @@ struct BwdTensorMaps {
 cudaError_t launch_bwd_dq_sm100(const BwdTensorMaps &tm, const float *lse, const float *abar, const float *go,
                                 const float *delta, float *dq, float *drho, int B, int H, int T, int d, int causal,
                                 int sm_count, int *work_counter, const DeviceCtl &ctl, cudaStream_t s);
-// Gradients of the prefill (mma.sync kernels): go, delta are [B*H*T] fp32
-// scratch; q, k, v, rho, dy bf16; y, o fp32 [B,H,T,d]; abar, lse fp32 [B,H,T];
-// dq, dk, dv, drho fp32 [B,H,T,d] (written).
-cudaError_t launch_bwd(const void *q, const void *k, const void *v, const void *rho, const void *dy, const float *y,
-                       const float *o, const float *abar, const float *lse, float *go, float *delta, float *dq,
-                       float *dk, float *dv, float *drho, int B, int H, int T, int d, int causal, const BwdTensorMaps &tm,
-                       int sm_count, int *work_counter, const DeviceCtl &ctl, cudaStream_t s);
+// Rows of the packed per-query statistics of the backward per head: T rounded up to 64.
+inline int bwd_tpad(int T) { return (T + 63) / 64 * 64; }
+// dk and dv (fp32, [B,H,T,d]) on tcgen05 (bwd_dkdv_sm100.cu); stats: float4
+// [B*H*Tpad] of (lse log2 e, abar, go, delta) per query, padding rows
+// (+inf, 0, 0, 0); tm: q, rho, dY with 64-row boxes, k and v with 128-row boxes.
+cudaError_t launch_bwd_dkdv_sm100(const BwdTensorMaps &tm, const void *stats, float *dk, float *dv, int B, int H, int T,
+                                  int d, int causal, int sm_count, int *work_counter, const DeviceCtl &ctl,
+                                  cudaStream_t s);
+// Gradients of the prefill: go, delta are [B*H*T] fp32 scratch, st4 is
+// [B*H*bwd_tpad(T)] float4 scratch, counters two ints of scratch; tm_dq and
+// tm_dkdv the tensor maps of the two gradient kernels.
+cudaError_t launch_bwd(const void *dy, const float *y, const float *o, const float *abar, const float *lse, float *go,
+                       float *delta, void *st4, float *dq, float *dk, float *dv, float *drho, int B, int H, int T, int d,
+                       int causal, const BwdTensorMaps &tm_dq, const BwdTensorMaps &tm_dkdv, int sm_count,
+                       int *counters, const DeviceCtl &ctl, cudaStream_t s);
 
 }  // namespace plx
