@@ -609,8 +609,8 @@ def measure_extras(args, stream, barrier, world, peaks, pc, dpq, dpk, dpv, yp, l
                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                         "frac": round(b_flops / (b_ms * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)},
            "fwd_train_ms": round(tr_ms, 4),
-           "note": "parallax_bwd (mma.sync kernels; scores recomputed in both, 11 products executed per pair) "
-                   "after parallax_fwd_train on the prefill shape; flops count 8 GEMMs of 2d per pair"}
+           "note": "parallax_bwd (tcgen05 dq/drho and dk/dv kernels; S, A, G recomputed in both, 11 products "
+                   "executed per pair) after parallax_fwd_train on the prefill shape; flops count 8 GEMMs of 2d per pair"}
     del dpr, ddy, fwd_state
     return {"decode_paged": paged, "softmax_only_fwd": smx, "fwd_fused": fused, "bwd": bwd,
             "softmax_decode": softmax_decode}

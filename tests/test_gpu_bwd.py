@@ -76,3 +76,18 @@ def test_bwd_zero_probe_matches_softmax_attention_gradients():
     cs = max(np.abs(r).max() for r in ref)
     for name, mine, r in zip(("dq", "dk", "dv", "drho"), g, ref):
         parity.assert_grad_parity(mine, r, 2, f"{name} rho=0", case_scale=cs)
+
+
+def test_bwd_b8_t4096_h16_two_heads_vs_oracle():
+    """The timed backward shape, B=8 H=16 T=4096 d=128 causal, in one call: the
+    gradients of the first and the last head against the oracle computed on
+    those heads alone (each head's gradients depend on that head only)."""
+    B, H, T, d = 8, 16, 4096, 128
+    q, k, v, rho, dy = _case(B, H, T, d, seed=71)
+    _, g = _run(q, k, v, rho, dy, True)
+    for b, h in ((0, 0), (B - 1, H - 1)):
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        ref = oracle.bwd(q.f64[sl], k.f64[sl], v.f64[sl], rho.f64[sl], dy.f64[sl], causal=True)
+        cs = max(np.abs(r).max() for r in ref)
+        for name, mine, r in zip(("dq", "dk", "dv", "drho"), g, ref):
+            parity.assert_grad_parity(mine[sl], r, 2, f"{name} B=8 T=4096 head ({b},{h})", case_scale=cs)
