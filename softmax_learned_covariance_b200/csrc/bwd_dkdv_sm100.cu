@@ -18,8 +18,11 @@
 // statistics (lse log2 e, abar, go, delta) arrive as one packed 16-byte row
 // per query beside the tile.
 //
-// TMEM: tile regions X0, X1 (64 columns each), W regions W0, W1 (32 columns
-// each; query tile t uses X(t mod 2) and W(t mod 2)), accumulators dV, dK.
+// TMEM: one 64-column region per score product (S^T, A^T, G^T), so the three
+// products of the next query tile can be issued as soon as the elementwise
+// warps have read this tile's (the next S^T while this tile's A^T is being
+// read, and so on); W regions W0, W1 (32 columns each, query tile t uses
+// W(t mod 2)); accumulators dV, dK.
 // Shared memory: K and V of the item, a 3-stage ring of (Q, R, dY, statistics)
 // per query tile.
 //
@@ -70,13 +73,12 @@ template <int D> struct GeoK {
     static_assert(QT_BYTES % 1024 == 0 && STAGE_BYTES % 1024 == 0, "1024-byte aligned tiles");
 };
 
-// TMEM: X0 [0, 64), X1 [64, 128), W0 [128, 160), W1 [160, 192), dV, dK.
-constexpr uint32_t COL_X0 = 0, COL_W0 = 128, COL_DV = 256, COL_DK = 384;
-__host__ __device__ constexpr uint32_t col_x(uint32_t t) { return COL_X0 + (t & 1) * BQ; }
+// TMEM: S^T [0, 64), A^T [64, 128), G^T [128, 192), W0 [192, 224), W1 [224, 256), dV, dK.
+constexpr uint32_t COL_S = 0, COL_A = 64, COL_G = 128, COL_W0 = 192, COL_DV = 256, COL_DK = 384;
 __host__ __device__ constexpr uint32_t col_w(uint32_t t) { return COL_W0 + (t & 1) * (BQ / 2); }
-// In X: the bf16 dZ^T of queries [16c, 16c + 16) in columns [16c, 16c + 8) and
-// their dA^T in the next 8 (the G columns of those queries).  In W: the bf16
-// W^T of queries [16c, 16c + 16) in columns [8c, 8c + 8).
+// In the G region: the bf16 dZ^T of queries [16c, 16c + 16) in columns
+// [16c, 16c + 8) and their dA^T in the next 8 (the G columns of those
+// queries).  In W: the bf16 W^T of queries [16c, 16c + 16) in columns [8c, 8c + 8).
 constexpr uint32_t DA_SHIFT = 8;
 
 constexpr uint32_t IDESC_SC = idesc_f16(1, 1, 0, 0, BK, BQ);                          // bf16 K-major x bf16 K-major
@@ -89,8 +91,8 @@ struct __align__(8) BarsK {
     uint64_t s_free, a_free;           // the elementwise warps have read S^T, A^T
     uint64_t w_full[2];                // per W region: W^T of its tile written
     uint64_t wv_done[2];               // per W region: dv products of its tile done
-    uint64_t p_full[2];                // per X region: dZ^T, dA^T of its tile written
-    uint64_t pv_done[2];               // per X region: dk products of its tile done
+    uint64_t p_full;                   // dZ^T, dA^T of the current tile written
+    uint64_t pv_done;                  // dk products of the current tile done
     uint64_t om_free;                  // the epilogue has read dV and dK
     uint64_t drain[2];
     uint64_t sched_full[SCHED], sched_empty[SCHED];
@@ -165,9 +167,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int x = 0; x < 2; ++x) {
             mbar_init(smem_u32(&bars->w_full[x]), NSOFT_WARPS);
             mbar_init(smem_u32(&bars->wv_done[x]), 1);
-            mbar_init(smem_u32(&bars->p_full[x]), NSOFT_WARPS);
-            mbar_init(smem_u32(&bars->pv_done[x]), 1);
         }
+        mbar_init(smem_u32(&bars->p_full), NSOFT_WARPS);
+        mbar_init(smem_u32(&bars->pv_done), 1);
         mbar_init(smem_u32(&bars->om_free), NSOFT_WARPS);
         mbar_init(smem_u32(&bars->drain[0]), 1);
         mbar_init(smem_u32(&bars->drain[1]), 1);
@@ -243,9 +245,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (st_armed[s] >= 0) mbar_wait_drain(smem_u32(&bars->st_full[s]), (uint32_t)st_armed[s], DRAIN_NS);
     } else if (warp == 1 && lane == 0) {
         // ============================================= score UMMA issuer ==
-        // Query tile t: S^T(t) into X(t mod 2) once the dk products of tile
-        // t - 2 are done with the region, A^T(t) once S^T(t) is read, G^T(t)
-        // once A^T(t) is read.
+        // Query tile t: S^T(t) once S^T(t - 1) has been read, A^T(t) once
+        // A^T(t - 1) has been read, G^T(t) once the dk products of tile t - 1
+        // are done with the G region (they read dZ^T, dA^T there).
         uint32_t tc = 0;
         bool ok = true;
         const uint64_t dk_ = sdesc_sw128(sbase + Gm::OFF_K, 16, 1024);
@@ -269,21 +271,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             for (int t = 0; t < it.nqt; ++t, ++tc) {
                 const int s = tc % RST;
                 if (!mbar_wait(smem_u32(&bars->st_full[s]), (tc / RST) & 1, wc)) { ok = false; break; }
-                if (tc >= 2 && !mbar_wait(smem_u32(&bars->pv_done[tc & 1]), ((tc - 2) >> 1) & 1, wc)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
                 const uint64_t st = dring + (uint64_t)(s * (Gm::STAGE_BYTES >> 4));
-                issue_scores(col_x(tc), dk_, st);                                         // S^T = K Q^T
+                if (tc > 0 && !mbar_wait(smem_u32(&bars->s_free), (tc - 1) & 1, wc)) { ok = false; break; }
+                tc_fence_after();
+                issue_scores(COL_S, dk_, st);                                             // S^T = K Q^T
                 tc_commit(smem_u32(&bars->s_full));
-                if (!mbar_wait(smem_u32(&bars->s_free), tc & 1, wc)) { ok = false; break; }
+                if (tc > 0 && !mbar_wait(smem_u32(&bars->a_free), (tc - 1) & 1, wc)) { ok = false; break; }
                 tc_fence_after();
-                issue_scores(col_x(tc), dk_, st + (uint64_t)(Gm::QT_BYTES >> 4));          // A^T = K R^T
+                issue_scores(COL_A, dk_, st + (uint64_t)(Gm::QT_BYTES >> 4));              // A^T = K R^T
                 tc_commit(smem_u32(&bars->a_full));
-                if (!mbar_wait(smem_u32(&bars->a_free), tc & 1, wc)) { ok = false; break; }
+                if (tc > 0 && !mbar_wait(smem_u32(&bars->pv_done), (tc - 1) & 1, wc)) { ok = false; break; }
                 tc_fence_after();
-                issue_scores(col_x(tc), dv_, st + (uint64_t)((2 * Gm::QT_BYTES) >> 4));    // G^T = V dY^T
+                issue_scores(COL_G, dv_, st + (uint64_t)((2 * Gm::QT_BYTES) >> 4));        // G^T = V dY^T
                 tc_commit(smem_u32(&bars->g_full));
                 if (t == it.nqt - 1) tc_commit(smem_u32(&bars->kv_empty));
             }
@@ -319,18 +318,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     umma_ts(tmem + COL_DV, tmem + col_w(tc) + 8 * kk, b, IDESC_GR, (t == 0 && kk == 0) ? 0u : 1u);
                 }
                 tc_commit(smem_u32(&bars->wv_done[tc & 1]));
-                if (!mbar_wait(smem_u32(&bars->p_full[tc & 1]), (tc >> 1) & 1, wc)) { ok = false; break; }
+                if (!mbar_wait(smem_u32(&bars->p_full), tc & 1, wc)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < BQ / 16; ++kk) {   // dk += dZ^T Q / sqrt(d) + dA^T R
                     const uint64_t bq = st + (uint64_t)((kk * 16 * 128) >> 4);
                     const uint64_t br = st + (uint64_t)((Gm::QT_BYTES + kk * 16 * 128) >> 4);
-                    const uint32_t zc = tmem + col_x(tc) + 16 * kk;
+                    const uint32_t zc = tmem + COL_G + 16 * kk;
                     umma_ts(tmem + COL_DK, zc, bq, IDESC_GR, (t == 0 && kk == 0) ? 0u : 1u);
                     umma_ts(tmem + COL_DK, zc + DA_SHIFT, br, IDESC_GR, 1u);
                 }
                 tc_commit(smem_u32(&bars->st_empty[s]));
-                tc_commit(smem_u32(&bars->pv_done[tc & 1]));
+                tc_commit(smem_u32(&bars->pv_done));
             }
         }
         tc_commit(smem_u32(&bars->drain[1]));
@@ -354,7 +353,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int key = it.kt * BK + r;
             for (int t = 0; t < it.nqt; ++t, ++tc) {
                 const int s = tc % RST;
-                const uint32_t xcol = tmem + lane_off + col_x(tc) + grp * QCOLS;
+                const uint32_t xcol = tmem + lane_off + grp * QCOLS;   // + COL_S, COL_A, COL_G
                 const uint32_t stq = sbase + Gm::OFF_RING + s * Gm::STAGE_BYTES + 3 * Gm::QT_BYTES + grp * QCOLS * 16;
                 const int qfirst = (it.q0t + t) * BQ + grp * QCOLS;   // this group's first query
                 if (!warp_wait(smem_u32(&bars->st_full[s]), (tc / RST) & 1, wc)) { ok = false; break; }
@@ -364,7 +363,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 float sv[QCOLS];
                 {
                     uint32_t sr[QCOLS];
-                    tmem_ld16(xcol, sr);
+                    tmem_ld16(xcol + COL_S, sr);
                     tmem_wait_ld();
                     tc_fence_before();
                     __syncwarp();
@@ -380,7 +379,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (!warp_wait(smem_u32(&bars->a_full), tc & 1, wc)) { ok = false; break; }
                 tc_fence_after();
                 uint32_t ar[QCOLS];
-                tmem_ld16(xcol, ar);
+                tmem_ld16(xcol + COL_A, ar);
                 tmem_wait_ld();
                 tc_fence_before();
                 __syncwarp();
@@ -410,7 +409,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 tc_fence_after();
                 {
                     uint32_t gv[QCOLS];
-                    tmem_ld16(xcol, gv);
+                    tmem_ld16(xcol + COL_G, gv);
                     tmem_wait_ld();
                     uint32_t zp[QCOLS / 2], dp[QCOLS / 2];
 #pragma unroll
@@ -427,18 +426,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         zp[i] = pack_bf16x2(z[0], z[1]);
                         dp[i] = pack_bf16x2(da[0], da[1]);
                     }
-                    tmem_st8(xcol, zp);
-                    tmem_st8(xcol + DA_SHIFT, dp);
+                    tmem_st8(xcol + COL_G, zp);
+                    tmem_st8(xcol + COL_G + DA_SHIFT, dp);
                     tmem_wait_st();
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[tc & 1]));
+                if (lane == 0) mbar_arrive(smem_u32(&bars->p_full));
             }
             if (!ok) break;
             // ---------------------------------------------- epilogue --
             // the item's last dk products are done (its dv products came first): dV, dK are final
-            if (!warp_wait(smem_u32(&bars->pv_done[(tc - 1) & 1]), ((tc - 1) >> 1) & 1, wc)) break;
+            if (!warp_wait(smem_u32(&bars->pv_done), (tc - 1) & 1, wc)) break;
             tc_fence_after();
             const bool store = key < T;
             const size_t row = (size_t)it.bh * T + (store ? key : 0);
