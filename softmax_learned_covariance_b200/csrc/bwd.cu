@@ -34,21 +34,26 @@ constexpr float LOG2E = 1.4426950408889634f;
 // ------------------------------------------------------------ row stats --
 // go_i = dY_i . o_i and delta_i = dY_i . y_i + abar_i go_i, one warp per row,
 // for rows padded to Tpad per head: go and delta go to [B*H*T] arrays (real
-// rows only) and a packed (lse_i log2 e, abar_i, go_i, delta_i) row to
-// st4 [B*H*Tpad]; padding rows get (+inf, 0, 0, 0), i.e. zero weights.
+// rows only) and (lse_i log2 e, abar_i, go_i, delta_i) to the packed
+// statistics: per head and 64-row block, the 64 values of each of the four in
+// turn (1 KB per block); padding rows get (+inf, 0, 0, 0), i.e. zero weights.
 template <int D>
 __global__ void __launch_bounds__(256) k_bwd_rowstats(const __nv_bfloat16 *__restrict__ dy, const float *__restrict__ o,
                                                      const float *__restrict__ y, const float *__restrict__ abar,
                                                      const float *__restrict__ lse, float *__restrict__ go,
-                                                     float *__restrict__ delta, float4 *__restrict__ st4, int T,
+                                                     float *__restrict__ delta, float *__restrict__ st, int T,
                                                      int Tpad, long prows) {
     const long prow = (long)blockIdx.x * 8 + threadIdx.x / 32;
     const int lane = threadIdx.x & 31;
     if (prow >= prows) return;
     const long bh = prow / Tpad;
     const int t = (int)(prow % Tpad);
+    float *blk = st + (prow - (t & 63)) * 4 + (t & 63);   // this row's slot in its block
     if (t >= T) {
-        if (lane == 0) st4[prow] = make_float4(INFINITY, 0.f, 0.f, 0.f);
+        if (lane == 0) {
+            blk[0] = INFINITY;
+            blk[64] = blk[128] = blk[192] = 0.f;
+        }
         return;
     }
     const long row = bh * T + t;
@@ -68,7 +73,10 @@ __global__ void __launch_bounds__(256) k_bwd_rowstats(const __nv_bfloat16 *__res
         const float ab = abar[row], dl = sy + ab * so;
         go[row] = so;
         delta[row] = dl;
-        st4[prow] = make_float4(lse[row] * LOG2E, ab, so, dl);
+        blk[0] = lse[row] * LOG2E;
+        blk[64] = ab;
+        blk[128] = so;
+        blk[192] = dl;
     }
 }
 
@@ -80,7 +88,7 @@ cudaError_t launch_t(const void *dy, const float *y, const float *o, const float
     const int Tpad = bwd_tpad(T);
     const long prows = (long)B * H * Tpad;
     k_bwd_rowstats<D><<<(unsigned)((prows + 7) / 8), 256, 0, s>>>((const __nv_bfloat16 *)dy, o, y, abar, lse, go, delta,
-                                                                   static_cast<float4 *>(st4), T, Tpad, prows);
+                                                                   static_cast<float *>(st4), T, Tpad, prows);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if ((e = launch_bwd_dq_sm100(tm_dq, lse, abar, go, delta, dq, drho, B, H, T, D, causal, sm_count, counters, ctl, s)))

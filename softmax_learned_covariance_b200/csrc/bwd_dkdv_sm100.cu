@@ -15,8 +15,9 @@
 // dZ^T / sqrt(d), dA^T (bf16) over the G columns they have read, and the
 // second issuing thread accumulates dv += W^T dY and dk += dZ^T Q + dA^T R in
 // TMEM (the Q, R and dY tiles read as MN-major B operands).  The per-query
-// statistics (lse log2 e, abar, go, delta) arrive as one packed 16-byte row
-// per query beside the tile.
+// statistics (lse log2 e, abar, go, delta) arrive beside the tile as 64 values
+// of each in turn, so a thread reads its 16 queries' values of one statistic
+// with four 16-byte loads.
 //
 // TMEM: one 64-column region per score product (S^T, A^T, G^T), so the three
 // products of the next query tile can be issued as soon as the elementwise
@@ -62,7 +63,7 @@ template <int D> struct GeoK {
     static constexpr int HALVES = D / 64;
     static constexpr int KV_BYTES = BK * D * 2;          // one 128-row bf16 tile
     static constexpr int QT_BYTES = BQ * D * 2;          // one 64-row bf16 tile
-    static constexpr int ST_BYTES = BQ * 16;             // packed statistics of a query tile
+    static constexpr int ST_BYTES = 4 * BQ * 4;          // statistics of a query tile: 4 x 64 floats
     static constexpr int STAGE_BYTES = 3 * QT_BYTES + ST_BYTES;   // Q | R | dY | statistics
     static constexpr int OFF_K = 0;
     static constexpr int OFF_V = OFF_K + KV_BYTES;
@@ -354,7 +355,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             for (int t = 0; t < it.nqt; ++t, ++tc) {
                 const int s = tc % RST;
                 const uint32_t xcol = tmem + lane_off + grp * QCOLS;   // + COL_S, COL_A, COL_G
-                const uint32_t stq = sbase + Gm::OFF_RING + s * Gm::STAGE_BYTES + 3 * Gm::QT_BYTES + grp * QCOLS * 16;
+                // this group's 16 values of statistic k at stq + k * 256 (lse log2 e, abar, go, delta)
+                const uint32_t stq = sbase + Gm::OFF_RING + s * Gm::STAGE_BYTES + 3 * Gm::QT_BYTES + grp * QCOLS * 4;
                 const int qfirst = (it.q0t + t) * BQ + grp * QCOLS;   // this group's first query
                 if (!warp_wait(smem_u32(&bars->st_full[s]), (tc / RST) & 1, wc)) { ok = false; break; }
                 // ---- s = exp(z - lse) of this key and the group's 16 queries ----
@@ -369,10 +371,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(smem_u32(&bars->s_free));
 #pragma unroll
-                    for (int c = 0; c < QCOLS; ++c) {
-                        const float l2 = ld_shared_f4(stq + c * 16).x;   // +inf for queries past T
-                        const bool vis = !causal || qfirst + c >= key;
-                        sv[c] = vis ? ex2(fmaf(__uint_as_float(sr[c]), sc, -l2)) : 0.f;
+                    for (int c4 = 0; c4 < QCOLS / 4; ++c4) {
+                        const float4 l2 = ld_shared_f4(stq + c4 * 16);   // +inf for queries past T
+                        const float l2v[4] = {l2.x, l2.y, l2.z, l2.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int c = 4 * c4 + e;
+                            const bool vis = !causal || qfirst + c >= key;
+                            sv[c] = vis ? ex2(fmaf(__uint_as_float(sr[c]), sc, -l2v[e])) : 0.f;
+                        }
                     }
                 }
                 // ---- a, then W^T = s (1 + abar - a) into the tile's W region ----
@@ -387,10 +394,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 {
                     uint32_t wp[QCOLS / 2];
 #pragma unroll
-                    for (int i = 0; i < QCOLS / 2; ++i) {
-                        const float ab0 = ld_shared_f4(stq + (2 * i) * 16).y, ab1 = ld_shared_f4(stq + (2 * i + 1) * 16).y;
-                        wp[i] = pack_bf16x2(sv[2 * i] * (1.f + ab0 - __uint_as_float(ar[2 * i])),
-                                            sv[2 * i + 1] * (1.f + ab1 - __uint_as_float(ar[2 * i + 1])));
+                    for (int c4 = 0; c4 < QCOLS / 4; ++c4) {
+                        const float4 ab = ld_shared_f4(stq + 256 + c4 * 16);
+                        const int c = 4 * c4;
+                        wp[2 * c4] = pack_bf16x2(sv[c] * (1.f + ab.x - __uint_as_float(ar[c])),
+                                                 sv[c + 1] * (1.f + ab.y - __uint_as_float(ar[c + 1])));
+                        wp[2 * c4 + 1] = pack_bf16x2(sv[c + 2] * (1.f + ab.z - __uint_as_float(ar[c + 2])),
+                                                     sv[c + 3] * (1.f + ab.w - __uint_as_float(ar[c + 3])));
                     }
                     // the region's previous tile has been consumed by its dv products
                     if (tc >= 2 && !warp_wait(smem_u32(&bars->wv_done[tc & 1]), ((tc - 2) >> 1) & 1, wc)) {
@@ -413,18 +423,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     tmem_wait_ld();
                     uint32_t zp[QCOLS / 2], dp[QCOLS / 2];
 #pragma unroll
-                    for (int i = 0; i < QCOLS / 2; ++i) {
-                        float z[2], da[2];
+                    for (int c4 = 0; c4 < QCOLS / 4; ++c4) {
+                        const float4 ab4 = ld_shared_f4(stq + 256 + c4 * 16), go4 = ld_shared_f4(stq + 512 + c4 * 16),
+                                     dl4 = ld_shared_f4(stq + 768 + c4 * 16);
+                        const float abv[4] = {ab4.x, ab4.y, ab4.z, ab4.w}, gov[4] = {go4.x, go4.y, go4.z, go4.w},
+                                    dlv[4] = {dl4.x, dl4.y, dl4.z, dl4.w};
+                        float z[4], da[4];
 #pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int c = 2 * i + e;
-                            const float4 st4 = ld_shared_f4(stq + c * 16);   // (lse log2 e, abar, go, delta)
+                        for (int e = 0; e < 4; ++e) {
+                            const int c = 4 * c4 + e;
                             const float a = __uint_as_float(ar[c]), g = __uint_as_float(gv[c]);
-                            z[e] = sv[c] * (fmaf(1.f + st4.y - a, g, a * st4.z) - st4.w) * inv_sqrt;
-                            da[e] = sv[c] * (st4.z - g);
+                            z[e] = sv[c] * (fmaf(1.f + abv[e] - a, g, a * gov[e]) - dlv[e]) * inv_sqrt;
+                            da[e] = sv[c] * (gov[e] - g);
                         }
-                        zp[i] = pack_bf16x2(z[0], z[1]);
-                        dp[i] = pack_bf16x2(da[0], da[1]);
+                        zp[2 * c4] = pack_bf16x2(z[0], z[1]);
+                        zp[2 * c4 + 1] = pack_bf16x2(z[2], z[3]);
+                        dp[2 * c4] = pack_bf16x2(da[0], da[1]);
+                        dp[2 * c4 + 1] = pack_bf16x2(da[2], da[3]);
                     }
                     tmem_st8(xcol + COL_G, zp);
                     tmem_st8(xcol + COL_G + DA_SHIFT, dp);

@@ -116,14 +116,15 @@ cudaError_t launch_bwd_dq_sm100(const BwdTensorMaps &tm, const float *lse, const
                                 int sm_count, int *work_counter, const DeviceCtl &ctl, cudaStream_t s);
 // Rows of the packed per-query statistics of the backward per head: T rounded up to 64.
 inline int bwd_tpad(int T) { return (T + 63) / 64 * 64; }
-// dk and dv (fp32, [B,H,T,d]) on tcgen05 (bwd_dkdv_sm100.cu); stats: float4
-// [B*H*Tpad] of (lse log2 e, abar, go, delta) per query, padding rows
-// (+inf, 0, 0, 0); tm: q, rho, dY with 64-row boxes, k and v with 128-row boxes.
+// dk and dv (fp32, [B,H,T,d]) on tcgen05 (bwd_dkdv_sm100.cu); stats: per head
+// and 64-query block the 64 values of lse log2 e, abar, go and delta in turn
+// (B*H*Tpad*4 floats), padding queries (+inf, 0, 0, 0); tm: q, rho, dY with
+// 64-row boxes, k and v with 128-row boxes.
 cudaError_t launch_bwd_dkdv_sm100(const BwdTensorMaps &tm, const void *stats, float *dk, float *dv, int B, int H, int T,
                                   int d, int causal, int sm_count, int *work_counter, const DeviceCtl &ctl,
                                   cudaStream_t s);
 // Gradients of the prefill: go, delta are [B*H*T] fp32 scratch, st4 is
-// [B*H*bwd_tpad(T)] float4 scratch, counters two ints of scratch; tm_dq and
+// [B*H*bwd_tpad(T)*4] fp32 scratch (the packed statistics), counters two ints of scratch; tm_dq and
 // tm_dkdv the tensor maps of the two gradient kernels.
 cudaError_t launch_bwd(const void *dy, const float *y, const float *o, const float *abar, const float *lse, float *go,
                        float *delta, void *st4, float *dq, float *dk, float *dv, float *drho, int B, int H, int T, int d,
