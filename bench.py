@@ -600,8 +600,9 @@ def measure_extras(args, stream, barrier, world, peaks, pc, dpq, dpk, dpv, yp, l
     with torch.cuda.stream(stream):
         fwd_state = plx.parallax_fwd_train(dpq, dpk, dpv, dpr, stream=stream)
         tr_ms = timed(lambda: plx.parallax_fwd_train(dpq, dpk, dpv, dpr, stream=stream), max(2, args.steps // 4))
+        grads = [torch.empty_like(fwd_state[0]) for _ in range(4)]
         b_ms = timed(lambda: plx.parallax_bwd(dpq, dpk, dpv, dpr, *fwd_state[:1], fwd_state[2], fwd_state[3],
-                                              fwd_state[1], ddy, stream=stream), max(2, args.steps // 4))
+                                              fwd_state[1], ddy, stream=stream, out=grads), max(2, args.steps // 4))
     assert plx.parallax_last_device_error(stream) == 0
     b_flops = 16 * pc["d"] * pairs   # dV, dK (two), dQ, dR and the three recomputed score products: 8 GEMMs
     bwd = {"ms": round(b_ms, 4), "tflops": round(b_flops / (b_ms * 1e-3) / 1e12, 2), "flops": b_flops,
@@ -611,7 +612,7 @@ def measure_extras(args, stream, barrier, world, peaks, pc, dpq, dpk, dpv, yp, l
            "fwd_train_ms": round(tr_ms, 4),
            "note": "parallax_bwd (tcgen05 dq/drho and dk/dv kernels; S, A, G recomputed in both, 11 products "
                    "executed per pair) after parallax_fwd_train on the prefill shape; flops count 8 GEMMs of 2d per pair"}
-    del dpr, ddy, fwd_state
+    del dpr, ddy, fwd_state, grads
     return {"decode_paged": paged, "softmax_only_fwd": smx, "fwd_fused": fused, "bwd": bwd,
             "softmax_decode": softmax_decode}
 

@@ -184,14 +184,23 @@ def parallax_fwd_train(q, k, v, rho, causal: bool = True, stream=None):
     return y, lse, o, abar
 
 
-def parallax_bwd(q, k, v, rho, y, o, abar, lse, dy, causal: bool = True, stream=None):
-    """Gradients (dq, dk, dv, drho), fp32, for an upstream dy (bf16, [B, H, T, d])."""
+def parallax_bwd(q, k, v, rho, y, o, abar, lse, dy, causal: bool = True, stream=None, out=None):
+    """Gradients (dq, dk, dv, drho), fp32, for an upstream dy (bf16, [B, H, T, d]).
+
+    ``out``: optional (dq, dk, dv, drho) fp32 [B, H, T, d] tensors to write into."""
     torch = _torch()
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (rho, "rho"), (y, "y"), (o, "o"), (abar, "abar"), (lse, "lse"),
                  (dy, "dy")):
         _need(t, n)
     B, H, T, d = q.shape
-    outs = [torch.empty((B, H, T, d), dtype=torch.float32, device=q.device) for _ in range(4)]
+    if out is None:
+        outs = [torch.empty((B, H, T, d), dtype=torch.float32, device=q.device) for _ in range(4)]
+    else:
+        outs = list(out)
+        for t, n in zip(outs, ("dq", "dk", "dv", "drho")):
+            _need(t, n)
+            if t.dtype != torch.float32 or tuple(t.shape) != (B, H, T, d):
+                raise ValueError(f"{n} must be float32 of shape {(B, H, T, d)}")
     st = lib().parallax_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(rho), _ptr(y), _ptr(o), _ptr(abar), _ptr(lse), _ptr(dy),
                             *(_ptr(t) for t in outs), B, H, T, d, int(bool(causal)), _dtype_code(q.dtype),
                             _stream(stream))
