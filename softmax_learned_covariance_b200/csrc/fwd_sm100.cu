@@ -39,13 +39,19 @@
 // sub-partition with four softmax warps, and every barrier wait or commit it
 // makes between UMMAs leaves the tensor pipe idle.  Two threads therefore
 // issue: one the score UMMAs S(j), A(j), one the P.V UMMAs, so a wait of one
-// chain never stalls the other.  TMEM holds four 128-column regions: X (S of
-// a tile, then its A), P (the fp16 P and P o A' of a tile), O and M.  The
-// softmax releases X as soon as it has loaded S, and again once it has loaded
-// A; the P region is free once the previous tile's P.V UMMAs are done.
+// chain never stalls the other.  TMEM holds two 128-column tile regions X0, X1
+// and the accumulators O and M.  Key tile G uses X(G mod 2): S(G) lands there,
+// then A(G) once the softmax has read S(G), and the softmax writes the fp16 P
+// and P o A' over the S/A columns it has read; the region takes tile G + 2's S
+// once the P.V UMMAs of tile G are done, so the next tile's S never waits for
+// this tile's softmax.  While the four groups exchange their row maxima, each
+// forms P with the current reference when its own scores do not move it (and
+// rescales P if another group's do).
 // (Measured and dropped: a 768-thread layout with a separate epilogue
-// warpgroup, and converting V inside the kernel; both slowed the softmax
-// warps, which set the pace, more than they saved.)
+// warpgroup; converting V inside the kernel; two softmax teams of 8 warps on
+// alternate tiles; y through a shared-memory staging tile and TMA stores; the
+// epilogue deferred past the next item's first tile.  Each slowed the softmax
+// warps, which set the pace, or added register spills, more than it saved.)
 //
 // Roles (640 threads, one CTA per SM, persistent over (head, query tile)
 // items taken longest-first from an atomic work counter):
