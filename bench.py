@@ -378,7 +378,8 @@ def run_ours(args, rank, world):
         step()
     assert plx.parallax_last_device_error() == 0
     nsplit_units = plx.parallax_decode_workspace_bytes(dc["B"], dc["H"], dc["Tcap"], dc["d"])
-    launches_per_step = (2 if nsplit_units > 0 else 1) + 1 + 1   # decode (+ combine), rho_proj, fwd
+    # decode split (+ combine), rho_proj, and fwd's two kernels (V to block-scaled fp16, then k_fwd)
+    launches_per_step = (2 if nsplit_units > 0 else 1) + 1 + 2
 
     clocks = ClockSampler(dev.index)
     clocks.start()
