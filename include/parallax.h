@@ -160,10 +160,12 @@ PARALLAX_API int parallax_fwd_train(const void *q, const void *k, const void *v,
  *   y, o, abar, lse  : the outputs of parallax_fwd_train on the same inputs.
  *   dq, dk, dv, drho : [B, H, T, d] fp32 (written, not accumulated).
  *   d in {64, 128}; B * H <= 65535; in_dtype must be BF16.
- * Warp-level tensor-core kernels (mma.sync): one over query blocks for dq and
- * drho, one over key blocks for dk and dv, both recomputing the scores, so no
- * gradient is accumulated with atomics and the result is deterministic.
- * Scratch: 8 bytes per row (see the conventions above).
+ * tcgen05 tensor-core kernels: one over 128-query tiles for dq and drho, one
+ * over 128-key tiles for dk and dv, both recomputing the scores, so no gradient
+ * is accumulated with atomics and the result is deterministic.
+ * Scratch (see the conventions above): 256 bytes of work counters, 8 bytes per
+ * row (g.o and delta), and 16 bytes per row of packed per-query statistics with
+ * T rounded up to a multiple of 64 per head.
  */
 PARALLAX_API int parallax_bwd(const void *q, const void *k, const void *v, const void *rho, const float *y,
                               const float *o, const float *abar, const float *lse, const void *dy, float *dq,

@@ -351,7 +351,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint64_t dq = sdesc_sw128(sbase + Gm::OFF_Q, 16, 1024);
         const uint64_t dr = sdesc_sw128(sbase + Gm::OFF_R, 16, 1024);
         const uint64_t dk = sdesc_sw128(sbase + Gm::OFF_K, 16, 1024);   // stage s: + s * K_BYTES / 16
-        // fused probe: R[128 x d] += X chunk (K-major) x W_R chunk (MN-major) into the P region
+        // fused probe: R[128 x d] += X chunk (K-major) x W_R chunk (MN-major) into a tile region
         constexpr uint32_t IDESC_R = idesc_f16(1, 1, 0, 1, BM, D);
         auto issue_probe_chunk = [&](uint32_t dcol, uint32_t stage_addr, bool first) {
 #pragma unroll
