@@ -27,11 +27,18 @@
 // merged at the end and written as the same partials (or y) as the split
 // kernel, so the split combine applies unchanged.
 //
-// Occupancy over depth (measured, B=64 Hq=32 Hkv=8 ctx 4096): a 3-stage ring
-// at 2 CTAs per SM (210 registers, 96 KB each) streamed 0.73 of HBM; a
-// 2-stage ring at 3 CTAs per SM (registers capped at 170, no spills) 0.84,
-// and 0.92 with one query head per KV head; 4 CTAs per SM (128 registers)
-// spilled and fell to 0.69.
+// A 16-token tile starts on a multiple of 16 tokens and a page holds at least
+// 16, so the tile's rows share one page: its block-table entry is read once,
+// one iteration before the tile is copied, and that load overlaps the current
+// tile's arithmetic (read per row and chunk, just before the copies, it held
+// every copy back by a dependent global load: 0.85 of HBM at B=64 Hq=32 Hkv=8
+// ctx 4096 against 0.92 now, and 0.83 against 0.98 at B=256 with 16-token pages).
+//
+// Occupancy over depth (measured, B=64 Hq=32 Hkv=8 ctx 4096, before the page
+// read moved ahead): a 3-stage ring at 2 CTAs per SM (210 registers, 96 KB
+// each) streamed 0.73 of HBM; a 2-stage ring at 3 CTAs per SM (registers
+// capped at 170, no spills) 0.84, and 0.92 with one query head per KV head; 4
+// CTAs per SM (128 registers) spilled and fell to 0.69.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <math.h>
@@ -175,10 +182,19 @@ __global__ void __launch_bounds__(WARPS * 32, MIN_CTAS) k_decode_gqa(
         float m_run = -INFINITY, l_run = 0.f, ab_run = 0.f;
 
         uint8_t *ring = smem + warp * STAGES * GqaSmem<D>::STAGE_BYTES;
-        // copy tile i of this warp (tokens t0 + 16 i ..) into stage s; rows past t1 are zero-filled
-        auto issue = [&](int i, int s) {
+        // page of tile i: its 16 tokens start on a multiple of 16 and pages hold
+        // at least 16 tokens, so they share one page; i < ntiles keeps the
+        // table index below max_pages
+        auto page_of = [&](int i) -> int {
+            return pg.table[(size_t)b * pg.max_pages + ((t0 + i * TILE) >> pg.pshift)];
+        };
+        // copy tile i of this warp (tokens t0 + 16 i ..) from page `id` into stage s;
+        // rows past t1 are zero-filled
+        auto issue = [&](int i, int s, int id) {
             uint8_t *kt = ring + s * GqaSmem<D>::STAGE_BYTES;
             uint8_t *vt = kt + TILE * D * 2;
+            const bool bad = id < 0 || id >= pg.num_pages;
+            if (bad) atomicExch(err, PARALLAX_ERR_DEVICE_INDEX);
 #pragma unroll
             for (int k = 0; k < TILE * NCH / 32; ++k) {
                 const int idx = lane + 32 * k;
@@ -187,10 +203,7 @@ __global__ void __launch_bounds__(WARPS * 32, MIN_CTAS) k_decode_gqa(
                 const __nv_bfloat16 *ksrc = kp, *vsrc = vp;
                 uint32_t bytes = 0;
                 if (t < t1) {
-                    int id = pg.table[(size_t)b * pg.max_pages + (t >> pg.pshift)];
-                    if (id < 0 || id >= pg.num_pages) {
-                        atomicExch(err, PARALLAX_ERR_DEVICE_INDEX);
-                    } else {
+                    if (!bad) {
                         const size_t off = (((size_t)id * pg.Hkv + kvh) * (size_t)(pmask + 1) + (t & pmask)) * D + ch * 8;
                         ksrc = kp + off;
                         vsrc = vp + off;
@@ -205,14 +218,18 @@ __global__ void __launch_bounds__(WARPS * 32, MIN_CTAS) k_decode_gqa(
         // this warp's tiles are i = warp + WARPS k; tile k lives in stage k % STAGES
 #pragma unroll
         for (int k = 0; k < STAGES - 1; ++k) {
-            if (warp + WARPS * k < ntiles) issue(warp + WARPS * k, k);
+            if (warp + WARPS * k < ntiles) issue(warp + WARPS * k, k, page_of(warp + WARPS * k));
             cp_async_commit();
         }
+        // the page of the next tile to copy is read one iteration ahead, so its
+        // load overlaps this iteration's arithmetic
+        int id_next = warp + WARPS * (STAGES - 1) < ntiles ? page_of(warp + WARPS * (STAGES - 1)) : 0;
         int s = 0;
         for (int i = warp, k = 0; i < ntiles; i += WARPS, ++k, s = (s + 1 == STAGES) ? 0 : s + 1) {
             const int inext = i + WARPS * (STAGES - 1);
-            if (inext < ntiles) issue(inext, (s + STAGES - 1) % STAGES);   // the stage computed last iteration
+            if (inext < ntiles) issue(inext, (s + STAGES - 1) % STAGES, id_next);   // the stage computed last iteration
             cp_async_commit();
+            if (inext + WARPS < ntiles) id_next = page_of(inext + WARPS);
             cp_async_wait<STAGES - 1>();
             __syncwarp();
             const uint8_t *kt = ring + s * GqaSmem<D>::STAGE_BYTES;
