@@ -79,12 +79,19 @@ def decode_bytes(B, H, d, seqlens):
     return kv + B * H * d * 2 * 2 + B * H * d * 4
 
 
-# DRAM bytes per algorithmic byte of the decode kernel, from an ncu capture of
-# the same kernel at B=16 H=16 ctx 8192 (1.0739 GB read + 0.0099 GB written for
-# 1.0740 GB of K/V rows, q, rho and y).  Traffic grows in proportion to the
-# cached tokens read, so a launch's traffic is this ratio times its algorithmic
-# bytes.
-DECODE_TRAFFIC_RATIO = 1.0838 / 1.0740
+# DRAM bytes per algorithmic byte of the decode split kernel, from an ncu
+# capture of the default step's decode (B=64 H=16 ctx 4096: 2.148242 GB read +
+# 0.008331 GB written for 2.148532 GB of K/V rows, q, rho and y; the B=16
+# ctx 8192 capture gave 1.009).  Traffic grows in proportion to the cached
+# tokens read, so a launch's traffic is this ratio times its algorithmic bytes.
+DECODE_TRAFFIC_RATIO = (2.148242 + 0.008331) / 2.148532
+
+# DRAM bytes of one prefill forward kernel launch (ncu, dram__bytes_read.sum +
+# dram__bytes_write.sum of k_fwd) at the two prefill shapes the bench runs,
+# beside its algorithmic bytes (q, k, rho and the fp16 V read once, y written):
+# the K/V tiles are re-read from DRAM by the query tiles of a head whose
+# earlier reads have left L2.
+PREFILL_TRAFFIC = {(8, 4096): 3.934873e9 + 0.248365e9, (1, 32768): 4.051134e9 + 0.250774e9}
 
 
 def prefill_pairs(B, H, T, causal=True):
@@ -162,8 +169,10 @@ def run_profile_case(args):
     """Small single-kernel loops for ncu captures (inputs still larger than L2, a few GB at most).
 
     profile_fwd    : parallax_fwd, B=2 H=16 T=8192 d=128 causal (plus its rho input)
+    profile_fwd_b8 : parallax_fwd, B=8 H=16 T=4096 d=128 causal (the prefill of the default step)
     profile_fwd_long : parallax_fwd, B=1 H=16 T=32768 d=128 causal (the long prefill)
     profile_decode : parallax_decode, B=16 H=16 d=128, 8192-token cache
+    profile_decode_b64 : parallax_decode, B=64 H=16 d=128, 4096-token cache (the default step's decode)
     profile_rho    : parallax_rho_proj, x [2, 8192, 2048] @ W_R [2048, 2048]
     profile_paged  : parallax_decode_paged, B=64 Hq=32 Hkv=8, 64-token pages, ctx 4096 (1.07 GB)
     profile_bwd    : parallax_bwd, B=2 H=16 T=4096 d=128 causal (after one parallax_fwd_train)
@@ -175,19 +184,20 @@ def run_profile_case(args):
 
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    if args.workload in ("profile_fwd", "profile_fwd_long"):
-        B, T = (2, 8192) if args.workload == "profile_fwd" else (1, 32768)
-        q, k, v, r = (t.torch().to(dev) for t in inputs.fwd_bf16_inputs(B, 16, T, 128, seed=3 if B == 2 else 5))
+    if args.workload in ("profile_fwd", "profile_fwd_b8", "profile_fwd_long"):
+        B, T = {"profile_fwd": (2, 8192), "profile_fwd_b8": (8, 4096), "profile_fwd_long": (1, 32768)}[args.workload]
+        q, k, v, r = (t.torch().to(dev) for t in inputs.fwd_bf16_inputs(B, 16, T, 128, seed=5 if B == 1 else 3))
         y = torch.empty(q.shape, dtype=torch.float32, device=dev)
         call = lambda: plx.parallax_fwd(q, k, v, r, y=y, want_lse=False)
         work, unit = prefill_flops(B, 16, T, 128), "TFLOP/s"
-    elif args.workload == "profile_decode":
-        q, r, kc, vc, sl = inputs.decode_inputs(16, 16, 8192, 128, seed=2)
+    elif args.workload in ("profile_decode", "profile_decode_b64"):
+        B, ctx = (16, 8192) if args.workload == "profile_decode" else (64, 4096)
+        q, r, kc, vc, sl = inputs.decode_inputs(B, 16, ctx, 128, seed=2)
         q, r, kc, vc = (t.torch().to(dev) for t in (q, r, kc, vc))
         dsl = torch.from_numpy(sl).to(dev)
-        y = torch.empty((16, 16, 128), dtype=torch.float32, device=dev)
+        y = torch.empty((B, 16, 128), dtype=torch.float32, device=dev)
         call = lambda: plx.parallax_decode(q, r, kc, vc, dsl, y=y, want_lse=False)
-        work, unit = decode_bytes(16, 16, 128, sl), "TB/s"
+        work, unit = decode_bytes(B, 16, 128, sl), "TB/s"
     elif args.workload == "profile_paged":
         c = PAGED_CFG
         mp = c["ctx"] // c["page_size"]
@@ -474,7 +484,10 @@ def run_ours(args, rank, world):
                     "fwd": {"ms": round(fwd_ms, 4), "tflops": round(fwd_tfs / world, 2), "flops": p_flops,
                             "roofline": {"bound": "tensor", "achieved": round(fwd_tfs / world, 2), "peak": bf16,
                                          "unit": "TFLOP/s", "frac": round(fwd_tfs / world / bf16, 4),
-                                         "peak_note": f"{tag} dense bf16 (burst)"}},
+                                         "peak_note": f"{tag} dense bf16 (burst)",
+                                         "traffic": PREFILL_TRAFFIC.get((pc["B"], pc["T"])),
+                                         "traffic_unit": "bytes/launch (k_fwd)",
+                                         "algorithmic_bytes_per_launch": pc["B"] * pc["H"] * pc["T"] * pc["d"] * (4 * 2 + 4)}},
                     "rho_proj": {"ms": round(rp_ms, 4), "tflops": round(rp_tfs / world, 2), "flops": r_flops,
                                  "frac": round(rp_tfs / world / bf16, 4)},
                     "e2e": e2e_pre},
@@ -688,7 +701,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["default", "prefill_long", "sweep", "profile_fwd", "profile_decode",
-                                           "profile_rho", "profile_paged", "profile_fwd_long", "profile_bwd"],
+                                           "profile_rho", "profile_paged", "profile_fwd_long", "profile_bwd",
+                                           "profile_fwd_b8", "profile_decode_b64"],
                     default="default")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
