@@ -110,56 +110,119 @@ def rho_proj_flops(B, T, d_model, H, d):
 # clocks sampled during the timed region
 # --------------------------------------------------------------------------- #
 class ClockSampler:
+    """SM clock and clock-event reasons of the benchmark's GPU while the timed
+    region runs.  NVML is read from a background thread every 5 ms (the timed
+    region can be a few tens of ms); only the samples taken between mark_start()
+    and mark_end() count (the nearest ones if none fell inside).  The device is
+    matched to the CUDA device by PCI bus id.  Without NVML, nvidia-smi at its
+    shortest interval is the fallback.  Read-only: no setting is changed."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
+        self.samples = []          # (host time, sm MHz, max MHz, set of reasons)
+        self.t0 = self.t1 = None
+        self.thread = None
         self.proc = None
-        self.path = None
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.gpu)
+        try:
+            bus = "%04x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
 
     def start(self):
+        import threading
         try:
-            fd, self.path = tempfile.mkstemp(prefix=f"parallax_clocks_{self.gpu}_", suffix=".csv")
-            self.f = os.fdopen(fd, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+            nv, h = self._nvml_handle()
+            get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons",
+                                  getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons", None))
+            bits = [(name, getattr(nv, attr)) for name, attr in self.REASONS]
+            smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            self.stop_flag = False
 
-    def stop(self):
-        if self.proc is None:
-            return None
+            def loop():
+                while not self.stop_flag:
+                    try:
+                        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                        r = get_reasons(h) if get_reasons else 0
+                        self.samples.append((time.perf_counter(), float(sm), float(smax),
+                                             {n for n, b in bits if r & b}))
+                    except Exception:
+                        pass
+                    time.sleep(0.005)
+
+            self.thread = threading.Thread(target=loop, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.thread = None
+            try:
+                fd, self.path = tempfile.mkstemp(prefix=f"parallax_clocks_{self.gpu}_", suffix=".csv")
+                self.f = os.fdopen(fd, "w")
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                     "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+            except Exception:
+                self.proc = None
+
+    def mark_start(self):
+        self.t0 = time.perf_counter()
+
+    def mark_end(self):
+        self.t1 = time.perf_counter()
+
+    def _from_smi(self):
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
         self.f.close()
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        names = [n for n, _ in self.REASONS]
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
+                self.samples.append((None, float(parts[1]), float(parts[2]),
+                                     {n for n, v in zip(names, parts[5:9]) if v.lower() == "active"}))
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
         try:
             os.unlink(self.path)
         except OSError:
             pass
-        if not sm:
+
+    def stop(self):
+        time.sleep(0.02)   # a sample or two after the region ends
+        if self.thread is not None:
+            self.stop_flag = True
+            self.thread.join(timeout=2)
+        elif self.proc is not None:
+            self._from_smi()
+        if not self.samples:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        inside = [x for x in self.samples if x[0] is not None and self.t0 is not None and self.t0 <= x[0] <= self.t1]
+        source = "nvml, 5 ms" if self.thread is not None else "nvidia-smi, 100 ms"
+        if not inside:   # nothing inside: the samples nearest to the region
+            mid = None if self.t0 is None else (self.t0 + (self.t1 or self.t0)) / 2
+            key = (lambda x: abs(x[0] - mid)) if mid is not None and self.samples[0][0] is not None else None
+            inside = sorted(self.samples, key=key)[:3] if key else self.samples
+        return {"sm_mhz": statistics.median(x[1] for x in inside), "sm_max_mhz": inside[0][2],
+                "reasons": sorted(set().union(*(x[3] for x in inside))), "samples": len(inside),
+                "source": source}
 
 
 # --------------------------------------------------------------------------- #
@@ -397,11 +460,13 @@ def run_ours(args, rank, world):
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
+    clocks.mark_start()
     start.record(stream)
     for i in range(args.steps):
         step(evs[i])
     end.record(stream)
     barrier()
+    clocks.mark_end()
     clk = clocks.stop()
     assert plx.parallax_last_device_error() == 0
     total_ms = start.elapsed_time(end)
