@@ -699,27 +699,20 @@ def measure_extras(args, stream, barrier, world, peaks, pc, dpq, dpk, dpv, yp, l
 # --------------------------------------------------------------------------- #
 # reference arm: the fp64 oracle on host cores, bounded samples of the same workloads
 # --------------------------------------------------------------------------- #
-def oracle_sample(budget_s=12.0):
-    import oracle
+def _oracle_decode_sample():
+    """The first 4 sequences of the decode step (64 of its 1024 heads), same recipe and seed, as fp64."""
     from softmax_learned_covariance_b200 import inputs
 
-    cores = oracle.max_threads()
     dc = DECODE_CFG
-    # the first 4 sequences of the decode step (64 of its 1024 heads), same recipe and seed
     nbs = 4
     q, rho, kc, vc, sl = inputs.decode_inputs(nbs, dc["H"], dc["Tcap"], dc["d"], seed=2)
-    qf, rf, kf, vf = q.f64, rho.f64, kc.f64, vc.f64
-    t0 = time.perf_counter()
-    reps = 0
-    while True:
-        oracle.decode(qf, rf, kf, vf, sl)
-        reps += 1
-        if time.perf_counter() - t0 > budget_s / 2:
-            break
-    dt = (time.perf_counter() - t0) / reps
-    dec_tbs = decode_bytes(nbs, dc["H"], dc["d"], sl) / dt / 1e12
-    dec_sample = f"{nbs * dc['H']} of the {dc['B'] * dc['H']} heads x {dc['Tcap']} tokens, x{reps}"
-    # the same oracle on one thread, on the first sequence (16 heads)
+    return (q.f64, rho.f64, kc.f64, vc.f64, sl), nbs
+
+
+def _oracle_decode_1thread(oracle, args_f64):
+    """The oracle decode on one thread, on the first sequence (16 heads): TB/s."""
+    qf, rf, kf, vf, sl = args_f64
+    cores = oracle.max_threads()
     oracle.set_threads(1)
     try:
         t0 = time.perf_counter()
@@ -727,7 +720,12 @@ def oracle_sample(budget_s=12.0):
         dt1 = time.perf_counter() - t0
     finally:
         oracle.set_threads(cores)
-    dec_tbs_1t = decode_bytes(1, dc["H"], dc["d"], sl[:1]) / dt1 / 1e12
+    return decode_bytes(1, DECODE_CFG["H"], DECODE_CFG["d"], sl[:1]) / dt1 / 1e12
+
+
+def _oracle_prefill_sample(oracle):
+    """The oracle prefill on every 8th causal row of one T=4096 head: TFLOP/s and a description."""
+    from softmax_learned_covariance_b200 import inputs
 
     pc = PREFILL_CFG
     pq, pk, pv, pr = inputs.fwd_bf16_inputs(1, 1, pc["T"], pc["d"], seed=3)
@@ -737,17 +735,57 @@ def oracle_sample(budget_s=12.0):
     dt = time.perf_counter() - t0
     pairs = int(np.sum(rows + 1))
     pre_tfs = 8 * pc["d"] * pairs / dt / 1e12
-    pre_sample = f"{rows.size} causal rows (every 8th) of one T={pc['T']} head, {pairs} pairs, {pairs / dt:.3e} pairs/s"
+    return pre_tfs, f"{rows.size} causal rows (every 8th) of one T={pc['T']} head, {pairs} pairs, {pairs / dt:.3e} pairs/s"
+
+
+def oracle_sample(budget_s=12.0):
+    """The oracle on a bounded sample of the step, timed for about budget_s / 2 on all host cores."""
+    import oracle
+
+    cores = oracle.max_threads()
+    args_f64, nbs = _oracle_decode_sample()
+    dc = DECODE_CFG
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.decode(*args_f64)
+        reps += 1
+        if time.perf_counter() - t0 > budget_s / 2:
+            break
+    dt = (time.perf_counter() - t0) / reps
+    sl = args_f64[4]
+    dec_tbs = decode_bytes(nbs, dc["H"], dc["d"], sl) / dt / 1e12
+    dec_sample = f"{nbs * dc['H']} of the {dc['B'] * dc['H']} heads x {dc['Tcap']} tokens, x{reps}"
+    dec_tbs_1t = _oracle_decode_1thread(oracle, args_f64)
+    pre_tfs, pre_sample = _oracle_prefill_sample(oracle)
     return cores, dec_tbs, dec_sample, pre_tfs, pre_sample, dec_tbs_1t
 
 
 def run_reference(args, rank, world):
+    """The oracle as it stands, on the host cores: W untimed and K timed steps, each one oracle decode
+    of the same bounded sample of the decode step (64 of its 1024 heads, the full 4096-token cache);
+    the value is that sample's algorithmic bytes over the mean step time.  The 1-thread figure and the
+    prefill sample are measured once, after the timed steps."""
     if rank != 0:
         return None
-    cores, dec_tbs, dec_sample, pre_tfs, pre_sample, dec_1t = oracle_sample()
+    import oracle
+
+    cores = oracle.max_threads()
+    args_f64, nbs = _oracle_decode_sample()
+    dc = DECODE_CFG
+    for _ in range(args.warmup):
+        oracle.decode(*args_f64)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.decode(*args_f64)
+    dt = (time.perf_counter() - t0) / args.steps
+    dec_tbs = decode_bytes(nbs, dc["H"], dc["d"], args_f64[4]) / dt / 1e12
+    dec_sample = f"{nbs * dc['H']} of the {dc['B'] * dc['H']} heads x {dc['Tcap']} tokens per step"
+    dec_1t = _oracle_decode_1thread(oracle, args_f64)
+    pre_tfs, pre_sample = _oracle_prefill_sample(oracle)
     line = {
         "metric": METRIC, "value": dec_tbs, "unit": "TB/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
         "config": {"workload": "decode step B=64 H=16 d=128 ctx=4096 (headline) + prefill B=8 T=4096 H=16 d=128",
                    "decode": dict(DECODE_CFG), "prefill": dict(PREFILL_CFG)},
