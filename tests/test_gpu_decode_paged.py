@@ -27,7 +27,7 @@ def _run(args, out_dtype=torch.float32, expect_err=0):
 
 
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("page_size", [16, 64, 256])
+@pytest.mark.parametrize("page_size", [16, 32, 64, 128, 256])
 @pytest.mark.parametrize("group", [1, 2, 4])
 def test_paged_grouped_small(group, page_size, d):
     B, Hkv = 4, 2
