@@ -31,9 +31,11 @@
  *     PARALLAX_ERR_DEVICE_INDEX there, and a non-finite prefill output
  *     PARALLAX_ERR_DEVICE_RANGE.  Read (and clear) it with
  *     parallax_last_device_error().
- *   - Scratch.  A call that needs scratch device memory (parallax_fwd on the
- *     tensor-core path: a work counter and a block-scaled fp16 copy of V;
- *     parallax_decode and parallax_decode_paged: the split partials) takes it
+ *   - Scratch.  A call that needs scratch device memory (parallax_fwd and its
+ *     variants on the tensor-core path: a work counter and a block-scaled fp16
+ *     copy of V; parallax_decode, parallax_softmax_decode and
+ *     parallax_decode_paged: the split partials; parallax_bwd: its work
+ *     counters and per-row statistics) takes it
  *     for that call alone from a library-owned, per-device stream-ordered
  *     memory pool
  *     (cudaMallocFromPoolAsync on `stream`) and returns it with cudaFreeAsync
